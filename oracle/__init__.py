@@ -1,0 +1,65 @@
+"""fp64 CPU oracle for the GPTQ layer pass and its intrinsic-LoRA variant.
+
+TEST INFRASTRUCTURE ONLY. This package is the slow, plain, obviously correct
+statement of what the CUDA path must compute. It is imported only by the test
+suite, by ``__graft_entry__.smoke()`` (to check one small run) and by the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py``. The product path
+never imports, links or calls anything in here, and nothing in here imports
+the product package: the two share no code. Inputs reach both from the
+``datagen`` module, which holds none of the method's arithmetic.
+
+Everything is float64 NumPy. Every function cites the page and section whose
+statement it follows. Where the pages leave a step open, the function says
+which reading it takes.
+
+Parity status of each function (what pins it; see tests/test_oracle_*.py):
+
+==============================  ==================================================
+hessian                         brute-force triple loop on tiny inputs
+damp                            closed form (mean of the diagonal)
+inverse_cholesky_upper          U^T U H = I, triangularity, and the Gram-Schmidt
+                                lengths of the QL factor of [X; mu I]
+minmax_grid                     hand-derived golden rows (tests/golden/grid_*.txt)
+sweep (plain)                   Babai nearest plane in data space (exact codes),
+                                round-to-nearest when X^T X = I, blocking
+                                invariance, brute force on tiny n, exact loss
+                                identity
+il_* (intrinsic LoRA)           r = 0 equals plain GPTQ bit for bit; literal
+                                eig+QR factor equals the Schur-complement route;
+                                R equals its closed-form conditional optimum;
+                                codes and R equal Babai on the augmented lattice;
+                                residual-based error bound
+pack_codes                      hand-derived golden words (tests/golden/pack_*.txt)
+==============================  ==================================================
+"""
+from .gptq import (
+    hessian,
+    damp,
+    inverse_cholesky_upper,
+    minmax_grid,
+    sweep,
+    sweep_blocked,
+    gptq_layer,
+    replay,
+    regularised_loss_rows,
+    data_loss_rows,
+)
+from .il import (
+    top_singular_directions,
+    augmented_gram,
+    il_hessian,
+    eig_qr_factor,
+    schur_factor_rows,
+    il_layer,
+    il_R_closed_form,
+)
+from .babai import ql_decomposition, babai_nearest_plane
+from .pack import pack_codes, unpack_codes
+
+__all__ = [
+    "hessian", "damp", "inverse_cholesky_upper", "minmax_grid", "sweep", "sweep_blocked",
+    "gptq_layer", "replay", "regularised_loss_rows", "data_loss_rows",
+    "top_singular_directions", "augmented_gram", "il_hessian", "eig_qr_factor",
+    "schur_factor_rows", "il_layer", "il_R_closed_form",
+    "ql_decomposition", "babai_nearest_plane", "pack_codes", "unpack_codes",
+]

@@ -1,0 +1,178 @@
+/*
+ * gptq.h — C ABI of the B200 (sm_100a) GPTQ layer-quantization library (libgptq.so).
+ *
+ * The library runs the GPTQ layer-wise quantization pass and its
+ * GPTQ-intrinsic-LoRA variant on one GPU:
+ *
+ *   gptq_hessian_accumulate   H += 2 X^T X over one chunk of calibration tokens
+ *   gptq_prepare_hinv         lambda = lambda_rel * mean(diag H); U upper with (H + lambda I)^-1 = U^T U
+ *   gptq_quantize_layer       column sweep of W onto per-group min-max grids with error feedback
+ *   gptq_il_quantize_layer    the same pass on the augmented calibration [X, X V_r]; returns Q, L = V_r, R
+ *
+ * Conventions shared by every entry point
+ *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);
+ *     X is k x n row-major (k calibration tokens). The pages write the layer as XW with W
+ *     stored in x out; this is its transpose. Columns are swept j = 0 .. n-1.
+ *   - Every pointer argument named as "device" must point to device memory of the current
+ *     device, owned by the caller; the library never allocates or frees device memory.
+ *     Scratch memory is passed in as `workspace` (size from gptq_workspace_size).
+ *   - Calls only enqueue work on `stream` (a cudaStream_t; NULL = the legacy default stream)
+ *     and return without synchronising. Argument errors are detected on the host and
+ *     returned at once (GPTQ_ERR_ARG / GPTQ_ERR_WORKSPACE); nothing is enqueued then.
+ *     Errors the device finds (a non-positive pivot, non-finite data, a timed-out wait)
+ *     are recorded in a sticky per-device status word: the first error wins and later
+ *     calls keep running on whatever data they get. Read and clear it with
+ *     gptq_sync_status(). A launch failure reported by the CUDA runtime is returned as
+ *     GPTQ_ERR_CUDA.
+ *   - There is no CPU fallback: every step runs in this library's CUDA kernels.
+ *   - Not thread-safe per device for overlapping calls that share a workspace.
+ */
+#ifndef GPTQ_H
+#define GPTQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GPTQ_API __attribute__((visibility("default")))
+#else
+#define GPTQ_API
+#endif
+
+typedef struct CUstream_st *gptq_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+    GPTQ_OK = 0,
+    GPTQ_ERR_ARG = -1,        /* bad pointer, size or option (host-side check) */
+    GPTQ_ERR_NOT_PD = -2,     /* a pivot <= 0 in the factorization (info: the column) */
+    GPTQ_ERR_NONFINITE = -3,  /* NaN or Inf in W or in diag(H) (info: the flat index) */
+    GPTQ_ERR_TIMEOUT = -4,    /* a bounded device-side wait gave up (info: the site) */
+    GPTQ_ERR_CUDA = -5,       /* the CUDA runtime refused a launch (see cudaGetLastError) */
+    GPTQ_ERR_WORKSPACE = -6   /* workspace pointer NULL, misaligned or too small */
+} gptq_status;
+
+typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
+
+typedef enum {
+    GPTQ_OP_HESSIAN = 0,
+    GPTQ_OP_PREPARE_HINV = 1,
+    GPTQ_OP_QUANTIZE = 2,
+    GPTQ_OP_IL_QUANTIZE = 3
+} gptq_op;
+
+/* Bytes of device workspace the entry point `op` needs for these sizes (0 if none).
+ * m, n: layer shape; r: intrinsic-LoRA rank (IL only, else 0); block_size: B.
+ * The workspace must be 256-byte aligned. Returns 0 for an unknown op. */
+GPTQ_API size_t gptq_workspace_size(int op, int64_t m, int64_t n, int r, int block_size);
+
+/* Human-readable name of a gptq_status value (static string, never NULL). */
+GPTQ_API const char *gptq_status_string(int status);
+
+/* Waits for `stream`, then returns the device status word of the current device
+ * (GPTQ_OK if no device-side error was recorded) and clears it. If `info` is not
+ * NULL it receives the error's detail (column / index / site; 0 if none). */
+GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info);
+
+/*
+ * H += 2 X^T X.
+ * GPTQ (encyclopedia article), "Technical approach": the quantizer is driven by the
+ * Hessian of the layer-wise squared error ||XW - XQ||^2, which is 2 X^T X.
+ *   H       device, n x n fp32 row-major, caller-owned; accumulated into (zero it before
+ *           the first chunk). On return both triangles hold the symmetric sum.
+ *   X       device, k x n row-major calibration chunk; x_dtype GPTQ_BF16 or GPTQ_F32.
+ *           The base address must be 16-byte aligned; for GPTQ_BF16, n % 8 == 0.
+ *   k, n    k >= 0 tokens (k == 0 is a no-op), 1 <= n <= 65536 features.
+ * Call it once per chunk of tokens; chunks are additive and may be of any length.
+ */
+GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64_t k, int64_t n,
+                            gptq_stream_t stream);
+
+/*
+ * lambda = lambda_rel * mean(diag H);  U upper triangular with (H + lambda I)^-1 = U^T U.
+ * GPTQ-2D (two-sided adaptive rounding), sections 2 and 4: the error feedback is read
+ * from a triangular factor of the inverse Gram matrix; Lattice Geometry of Neural
+ * Network Quantization, section 3.1: lambda regularisation keeps the basis independent.
+ * Computed as H + lambda I = Ubar Ubar^T (Cholesky from the last column backwards,
+ * Ubar upper) followed by U = Ubar^-1: the same U as chol -> inverse -> chol.
+ *   H          device, n x n fp32 (the raw 2 X^T X), read only; only the upper triangle
+ *              is read.
+ *   lambda_rel relative damping (> 0 recommended; >= 0 accepted).
+ *   U          device, n x n fp32, written: the upper triangle (diagonal included) holds
+ *              U; the strictly lower triangle is left zero.
+ *   lambda_out device, one fp32: the absolute lambda used.
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_PREPARE_HINV, 0, n, 0, 0) bytes.
+ * Device errors: GPTQ_ERR_NOT_PD (info = first column with pivot <= 0),
+ * GPTQ_ERR_NONFINITE (info = index of a non-finite diagonal entry of H).
+ */
+GPTQ_API int gptq_prepare_hinv(const float *H, int64_t n, float lambda_rel, float *U,
+                      float *lambda_out, void *workspace, size_t ws_bytes,
+                      gptq_stream_t stream);
+
+/*
+ * Quantize the columns of W one at a time with closed-form error feedback.
+ * GPTQ (encyclopedia article), "Technical approach" (column-wise greedy quantization,
+ * closed-form compensation of the remaining weights, per-group scales, 2/3/4-bit);
+ * GPTQ-2D, section 2 (GPTQ's lazy block update).
+ * For each column j: at a group start the grid of each row is taken from the current
+ * weights of the group (xmin = min(0, min w), xmax = max(0, max w), a zero range widened
+ * to [-1, 1], s = (xmax - xmin)/maxq, z = rint(-xmin/s)); v = w_j/s + z;
+ * c = clamp(rint(v), 0, maxq) (round half to even); e = (w_j - s(c - z)) / U_jj;
+ * the later columns of the row receive -e * U_{j, j+1:}. Inside a block of
+ * `block_size` columns this is done column by column; the columns after the block are
+ * updated once per block by W[:, after] -= Err * U[block, after].
+ *   W          device, m x n row-major, w_dtype GPTQ_BF16 or GPTQ_F32, read only.
+ *   U          device, n x n fp32 upper factor from gptq_prepare_hinv (row-major).
+ *   bits       2..8.  group_size: 0 (one group per row) or a divisor of n with
+ *              block_size % group_size == 0 or group_size % block_size == 0.
+ *   block_size 32, 64 or 128; n % block_size == 0.
+ *   codes      device, m x (n*bits/32) uint32 (n*bits % 32 == 0): along each row, code j
+ *              occupies bits [j*bits, j*bits + bits) of a little-endian bit stream cut
+ *              into 32-bit words, least significant bit first.
+ *   scales     device, m x G fp32, G = group_size ? n/group_size : 1.
+ *   zeros      device, m x G uint8 zero-points.
+ *   loss_out   device, m fp64 or NULL: per row sum_j e_j^2, which equals
+ *              (w - w_hat)^T (H + lambda I) (w - w_hat).
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size).
+ * Device errors: GPTQ_ERR_NONFINITE (info = flat index into W of a non-finite weight).
+ */
+GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
+                        int bits, int group_size, int block_size, uint32_t *codes,
+                        float *scales, uint8_t *zeros, double *loss_out, void *workspace,
+                        size_t ws_bytes, gptq_stream_t stream);
+
+/*
+ * GPTQ-intrinsic LoRA: quantize W against the augmented calibration X~ = [X, X V_r].
+ * GPTQ-intrinsic LoRA summary, "Method" part 2: V_r (= L) are the top-r right singular
+ * vectors of X; the pass runs on W~ = [W, 0] (r extra zero-initialised coordinates per
+ * row, placed after the n original ones and never quantized); the extra coordinates
+ * absorb the quantization error and end as R; the singular augmented Hessian is factored
+ * without a plain Cholesky of it. Here: V_r by subspace iteration on G = H/2 with a
+ * Rayleigh-Ritz step; H~ = 2 X~^T X~ + lambda~ I with lambda~ = lambda_rel * mean of
+ * the n + r diagonal entries of 2 X~^T X~; the first n rows of U~ (H~^-1 = U~^T U~)
+ * come from the Schur complement of the extra block, which is positive definite.
+ * With r == 0 this is gptq_prepare_hinv + gptq_quantize_layer.
+ *   H          device, n x n fp32 raw Hessian 2 X^T X (from gptq_hessian_accumulate).
+ *   r          0 <= r <= 128 and r < n.
+ *   L          device, n x r fp32 (V_r, columns sorted by decreasing eigenvalue, each
+ *              column's largest-magnitude entry positive); unused if r == 0.
+ *   R          device, r x m fp32 (row-major); unused if r == 0.
+ *   lambda_out device, one fp32: lambda~.
+ *   other arguments as in gptq_quantize_layer.
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_IL_QUANTIZE, m, n, r, block_size).
+ * Device errors as in gptq_prepare_hinv and gptq_quantize_layer.
+ */
+GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
+                           int r, int bits, int group_size, float lambda_rel, int block_size,
+                           uint32_t *codes, float *scales, uint8_t *zeros, float *L, float *R,
+                           float *lambda_out, double *loss_out, void *workspace,
+                           size_t ws_bytes, gptq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_H */

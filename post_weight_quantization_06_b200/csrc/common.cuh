@@ -1,0 +1,69 @@
+// Shared device helpers of libgptq: the sticky status word, launch checks, small math.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <math.h>
+
+#include "gptq.h"
+
+namespace gptq {
+
+// ---------------------------------------------------------------------------------------
+// Sticky device status word: the first device-side error wins; read and cleared by
+// gptq_sync_status(). One copy per device (a __device__ variable lives in every context).
+// ---------------------------------------------------------------------------------------
+struct DevStatus {
+    int code;
+    int pad;
+    long long info;
+};
+
+__device__ DevStatus g_status;
+
+__device__ __forceinline__ void report(int code, long long info) {
+    if (atomicCAS(&g_status.code, 0, code) == 0) {
+        atomicExch(reinterpret_cast<unsigned long long *>(&g_status.info),
+                   static_cast<unsigned long long>(info));
+    }
+}
+
+__device__ __forceinline__ bool finitef(float x) { return isfinite(x); }
+
+template <typename T> __device__ __forceinline__ float to_f32(T x);
+template <> __device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ float warp_min(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+inline int launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+#define GPTQ_CHECK_LAUNCH()                  \
+    do {                                     \
+        int _s = ::gptq::launch_status();    \
+        if (_s != GPTQ_OK) return _s;        \
+    } while (0)
+
+}  // namespace gptq

@@ -1,0 +1,149 @@
+// Generic fp32-accumulating SIMT GEMM: C = alpha * op(A) op(B) + beta * C, with optional
+// triangular structure. Used where a step is a small or awkward contraction (panel solves,
+// the fp32-input Hessian); large contractions go to the tcgen05 kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace gptq {
+
+template <typename TA, typename TB>
+struct GemmArgs {
+    int M, N, K;
+    const TA *A;
+    long long lda;
+    int ta;  // A(i,k) = ta ? A[k*lda + i] : A[i*lda + k]
+    const TB *B;
+    long long ldb;
+    int tb;  // B(k,j) = tb ? B[j*ldb + k] : B[k*ldb + j]
+    float *C;
+    long long ldc;
+    float alpha, beta;  // beta == 0: C is not read
+    int c_upper;        // write only C(i,j) with j >= i (tiles strictly below are skipped)
+    int a_upper;        // A(i,k) = 0 for k < i (storage there is not read)
+    int b_upper;        // B(k,j) = 0 for k > j (storage there is not read)
+};
+
+namespace simt {
+constexpr int BM = 128, BN = 128, BK = 16, NT = 256;
+}
+
+template <typename TA, typename TB>
+__global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
+    using namespace simt;
+    const int i0 = blockIdx.y * BM, j0 = blockIdx.x * BN;
+    if (p.c_upper && i0 >= j0 + BN) return;
+    __shared__ __align__(16) float As[BK][BM + 4];
+    __shared__ __align__(16) float Bs[BK][BN + 4];
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+    int kbeg = 0, kend = p.K;
+    if (p.a_upper) kbeg = max(kbeg, i0);
+    if (p.b_upper) kend = min(kend, j0 + BN);
+    kbeg = (kbeg / BK) * BK;
+
+    for (int k0 = kbeg; k0 < kend; k0 += BK) {
+#pragma unroll
+        for (int e = 0; e < (BM * BK) / NT; ++e) {
+            const int idx = tid + e * NT;
+            int r, kk;
+            if (p.ta) { kk = idx / BM; r = idx % BM; } else { r = idx / BK; kk = idx % BK; }
+            const int gi = i0 + r, gk = k0 + kk;
+            float v = 0.f;
+            if (gi < p.M && gk < kend && (!p.a_upper || gk >= gi))
+                v = to_f32(p.ta ? p.A[(long long)gk * p.lda + gi] : p.A[(long long)gi * p.lda + gk]);
+            As[kk][r] = v;
+        }
+#pragma unroll
+        for (int e = 0; e < (BN * BK) / NT; ++e) {
+            const int idx = tid + e * NT;
+            int c, kk;
+            if (p.tb) { c = idx / BK; kk = idx % BK; } else { kk = idx / BN; c = idx % BN; }
+            const int gj = j0 + c, gk = k0 + kk;
+            float v = 0.f;
+            if (gj < p.N && gk < kend && (!p.b_upper || gk <= gj))
+                v = to_f32(p.tb ? p.B[(long long)gj * p.ldb + gk] : p.B[(long long)gk * p.ldb + gj]);
+            Bs[kk][c] = v;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < BK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4 + 64]);
+            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4 + 64]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int gi = i0 + ty * 4 + (i & 3) + (i >> 2) * 64;
+        if (gi >= p.M) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int gj = j0 + tx * 4 + (j & 3) + (j >> 2) * 64;
+            if (gj >= p.N || (p.c_upper && gj < gi)) continue;
+            float *c = p.C + (long long)gi * p.ldc + gj;
+            *c = p.beta == 0.f ? p.alpha * acc[i][j] : fmaf(p.alpha, acc[i][j], p.beta * *c);
+        }
+    }
+}
+
+template <typename TA, typename TB>
+inline int gemm_simt(const GemmArgs<TA, TB> &p, cudaStream_t s) {
+    if (p.M <= 0 || p.N <= 0) return GPTQ_OK;
+    dim3 grid(ceil_div(p.N, simt::BN), ceil_div(p.M, simt::BM));
+    gemm_simt_kernel<TA, TB><<<grid, simt::NT, 0, s>>>(p);
+    return launch_status();
+}
+
+template <typename TA, typename TB>
+inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long lda, int ta,
+                                  const TB *B, long long ldb, int tb, float *C, long long ldc,
+                                  float alpha, float beta) {
+    GemmArgs<TA, TB> p;
+    p.M = M; p.N = N; p.K = K;
+    p.A = A; p.lda = lda; p.ta = ta;
+    p.B = B; p.ldb = ldb; p.tb = tb;
+    p.C = C; p.ldc = ldc;
+    p.alpha = alpha; p.beta = beta;
+    p.c_upper = 0; p.a_upper = 0; p.b_upper = 0;
+    return p;
+}
+
+// Copy the upper triangle of an n x n matrix onto its lower triangle (32x32 smem tiles).
+__global__ void mirror_upper_kernel(float *H, long long ld, int n) {
+    __shared__ float t[32][33];
+    const int bi = blockIdx.y, bj = blockIdx.x;  // destination tile (bi, bj) with bi >= bj
+    if (bi < bj) return;
+    const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+    for (int y = ty; y < 32; y += 8) {
+        const int r = bj * 32 + y, c = bi * 32 + tx;  // source: upper tile (bj, bi)
+        if (r < n && c < n) t[y][tx] = H[(long long)r * ld + c];
+    }
+    __syncthreads();
+    for (int y = ty; y < 32; y += 8) {
+        const int r = bi * 32 + y, c = bj * 32 + tx;
+        if (r < n && c < n && r > c) H[(long long)r * ld + c] = t[tx][y];
+    }
+}
+
+inline int mirror_upper(float *H, long long ld, int n, cudaStream_t s) {
+    dim3 grid(ceil_div(n, 32), ceil_div(n, 32));
+    mirror_upper_kernel<<<grid, dim3(32, 8), 0, s>>>(H, ld, n);
+    return launch_status();
+}
+
+}  // namespace gptq

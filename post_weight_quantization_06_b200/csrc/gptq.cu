@@ -1,0 +1,263 @@
+// libgptq: C ABI of the GPTQ / GPTQ-intrinsic-LoRA layer pass for sm_100a.
+// One translation unit: the kernels live in the included .cuh files.
+#include <cstring>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "factor.cuh"
+#include "quant.cuh"
+#include "il.cuh"
+
+namespace gptq {
+
+inline size_t align256(size_t b) { return (b + 255) & ~size_t(255); }
+
+// Carves typed sub-buffers out of the caller's workspace; with base == nullptr it only
+// counts, which is how gptq_workspace_size() and the call agree on the layout.
+struct Carver {
+    char *base;
+    size_t off = 0;
+    explicit Carver(void *b) : base(static_cast<char *>(b)) {}
+    template <typename T>
+    T *take(size_t count) {
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += align256(count * sizeof(T));
+        return p;
+    }
+};
+
+struct FactorWs {
+    float *A, *T;
+};
+inline FactorWs carve_factor(Carver &c, long long n) {
+    FactorWs w;
+    w.A = c.take<float>((size_t)n * n);
+    w.T = c.take<float>((size_t)FACTOR_NB * n);
+    return w;
+}
+
+struct QuantWs {
+    float *Wc, *Err;
+};
+inline QuantWs carve_quant(Carver &c, long long m, long long N, int B) {
+    QuantWs w;
+    w.Wc = c.take<float>((size_t)m * N);
+    w.Err = c.take<float>((size_t)m * B);
+    return w;
+}
+
+struct IlWs {
+    QuantWs q;
+    FactorWs f;
+    float *Uaug, *lam_dummy;
+    ILWork il;
+};
+inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
+    IlWs w;
+    w.q = carve_quant(c, m, n + r, B);
+    w.f = carve_factor(c, n);
+    w.Uaug = c.take<float>((size_t)n * (n + r));
+    w.lam_dummy = c.take<float>(1);
+    if (r > 0) {
+        const int p = il_block_p((int)n, r);
+        w.il.Y = c.take<float>((size_t)n * p);
+        w.il.Z = c.take<float>((size_t)n * p);
+        w.il.G = c.take<float>((size_t)p * p);
+        w.il.Gi = c.take<float>((size_t)p * p);
+        w.il.Tm = c.take<float>((size_t)p * p);
+        w.il.Qsel = c.take<float>((size_t)p * r);
+        w.il.ev = c.take<float>((size_t)p);
+        w.il.B12 = c.take<float>((size_t)n * r);
+        w.il.C = c.take<float>((size_t)r * r);
+        w.il.Ci = c.take<float>((size_t)r * r);
+        w.il.Y1 = c.take<float>((size_t)n * r);
+        w.il.Yr = c.take<float>((size_t)n * r);
+    } else {
+        std::memset(&w.il, 0, sizeof(w.il));
+    }
+    return w;
+}
+
+inline int check_ws(void *ws, size_t have, size_t need) {
+    if (need == 0) return GPTQ_OK;
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u) || have < need) return GPTQ_ERR_WORKSPACE;
+    return GPTQ_OK;
+}
+
+inline bool valid_quant_args(long long m, long long n, int bits, int gs, int B) {
+    if (m < 1 || n < 1 || m > (1LL << 30) || n > 65536) return false;
+    if (bits < 2 || bits > 8) return false;
+    if (B != 32 && B != 64 && B != 128) return false;
+    if (n % B) return false;
+    if ((n * bits) % 32) return false;
+    if (gs < 0) return false;
+    if (gs > 0) {
+        if (n % gs) return false;
+        if (B % gs && gs % B) return false;
+    }
+    return true;
+}
+
+template <typename TX>
+int hessian_simt(float *H, const TX *X, long long k, int n, cudaStream_t s) {
+    // H(upper) += 2 X^T X, then mirror; chunks of the token axis keep indices in range
+    const long long KCH = 1LL << 20;
+    for (long long t0 = 0; t0 < k; t0 += KCH) {
+        const int kc = (int)((k - t0) < KCH ? (k - t0) : KCH);
+        auto p = gemm_args<TX, TX>(n, n, kc, X + t0 * n, n, 1, X + t0 * n, n, 0, H, n, 2.f, 1.f);
+        p.c_upper = 1;
+        if (int st = gemm_simt(p, s)) return st;
+    }
+    return mirror_upper(H, n, n, s);
+}
+
+int prepare_hinv_impl(const float *H, int n, float lambda_rel, float *U, long long ldu,
+                      float *lambda_out, FactorWs &w, cudaStream_t s) {
+    damp_mean_kernel<<<1, 1024, 0, s>>>(H, n, n, lambda_rel, lambda_out);
+    GPTQ_CHECK_LAUNCH();
+    copy_damped_kernel<<<1184, 256, 0, s>>>(H, n, w.A, n, n, lambda_out);
+    GPTQ_CHECK_LAUNCH();
+    if (cudaMemsetAsync(U, 0, sizeof(float) * (size_t)n * ldu, s) != cudaSuccess) return GPTQ_ERR_CUDA;
+    return factor_ul_inverse(w.A, n, U, ldu, n, w.T, s);
+}
+
+int init_work(const void *W, int w_dtype, long long m, int n, float *Wc, long long ldw, int N,
+              cudaStream_t s) {
+    if (w_dtype == GPTQ_BF16)
+        init_work_kernel<__nv_bfloat16><<<1184, 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(W), m, n, Wc, ldw, N);
+    else
+        init_work_kernel<float><<<1184, 256, 0, s>>>(static_cast<const float *>(W), m, n, Wc, ldw, N);
+    return launch_status();
+}
+
+}  // namespace gptq
+
+using namespace gptq;
+
+extern "C" {
+
+GPTQ_API size_t gptq_workspace_size(int op, int64_t m, int64_t n, int r, int block_size) {
+    if (n < 1) return 0;
+    Carver c(nullptr);
+    switch (op) {
+        case GPTQ_OP_HESSIAN:
+            return 0;
+        case GPTQ_OP_PREPARE_HINV:
+            carve_factor(c, n);
+            return c.off;
+        case GPTQ_OP_QUANTIZE:
+            if (m < 1) return 0;
+            carve_quant(c, m, n, block_size > 0 ? block_size : 128);
+            return c.off;
+        case GPTQ_OP_IL_QUANTIZE:
+            if (m < 1 || r < 0) return 0;
+            carve_il(c, m, n, r, block_size > 0 ? block_size : 128);
+            return c.off;
+        default:
+            return 0;
+    }
+}
+
+GPTQ_API const char *gptq_status_string(int status) {
+    switch (status) {
+        case GPTQ_OK: return "GPTQ_OK";
+        case GPTQ_ERR_ARG: return "GPTQ_ERR_ARG: invalid argument";
+        case GPTQ_ERR_NOT_PD: return "GPTQ_ERR_NOT_PD: non-positive pivot in the factorization";
+        case GPTQ_ERR_NONFINITE: return "GPTQ_ERR_NONFINITE: NaN or Inf in the input";
+        case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT: a bounded device wait gave up";
+        case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA: CUDA runtime error";
+        case GPTQ_ERR_WORKSPACE: return "GPTQ_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        default: return "unknown gptq status";
+    }
+}
+
+GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GPTQ_ERR_CUDA;
+    DevStatus st;
+    if (cudaMemcpyFromSymbol(&st, g_status, sizeof(st)) != cudaSuccess) return GPTQ_ERR_CUDA;
+    DevStatus zero = {0, 0, 0};
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return GPTQ_ERR_CUDA;
+    if (info) *info = st.info;
+    return st.code;
+}
+
+GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64_t k, int64_t n,
+                                     gptq_stream_t stream) {
+    if (!H || !X || k < 0 || n < 1 || n > 65536) return GPTQ_ERR_ARG;
+    if (x_dtype != GPTQ_BF16 && x_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (k == 0) return GPTQ_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (x_dtype == GPTQ_BF16)
+        return hessian_simt(H, static_cast<const __nv_bfloat16 *>(X), k, (int)n, s);
+    return hessian_simt(H, static_cast<const float *>(X), k, (int)n, s);
+}
+
+GPTQ_API int gptq_prepare_hinv(const float *H, int64_t n, float lambda_rel, float *U,
+                               float *lambda_out, void *workspace, size_t ws_bytes,
+                               gptq_stream_t stream) {
+    if (!H || !U || !lambda_out || n < 1 || n > 65536) return GPTQ_ERR_ARG;
+    if (!(lambda_rel >= 0.f) || !isfinite(lambda_rel)) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_PREPARE_HINV, 0, n, 0, 0);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    Carver c(workspace);
+    FactorWs w = carve_factor(c, n);
+    return prepare_hinv_impl(H, (int)n, lambda_rel, U, n, lambda_out, w,
+                             reinterpret_cast<cudaStream_t>(stream));
+}
+
+GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
+                                 int bits, int group_size, int block_size, uint32_t *codes,
+                                 float *scales, uint8_t *zeros, double *loss_out,
+                                 void *workspace, size_t ws_bytes, gptq_stream_t stream) {
+    if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (!valid_quant_args(m, n, bits, group_size, block_size)) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(workspace);
+    QuantWs w = carve_quant(c, m, n, block_size);
+    if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
+    return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
+                       codes, scales, zeros, loss_out, w.Err, s);
+}
+
+GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n,
+                                    const float *H, int r, int bits, int group_size,
+                                    float lambda_rel, int block_size, uint32_t *codes,
+                                    float *scales, uint8_t *zeros, float *L, float *R,
+                                    float *lambda_out, double *loss_out, void *workspace,
+                                    size_t ws_bytes, gptq_stream_t stream) {
+    if (!W || !H || !codes || !scales || !zeros || !lambda_out) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (!valid_quant_args(m, n, bits, group_size, block_size)) return GPTQ_ERR_ARG;
+    if (r < 0 || r > IL_MAX_R || r >= n) return GPTQ_ERR_ARG;
+    if (r > 0 && (!L || !R)) return GPTQ_ERR_ARG;
+    if (!(lambda_rel >= 0.f) || !isfinite(lambda_rel)) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_IL_QUANTIZE, m, n, r, block_size);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(workspace);
+    IlWs w = carve_il(c, m, n, r, block_size);
+    const long long N = n + r;
+    if (r == 0) {
+        if (int st = prepare_hinv_impl(H, (int)n, lambda_rel, w.Uaug, n, lambda_out, w.f, s)) return st;
+    } else {
+        if (int st = il_top_eigvecs(H, n, (int)n, r, L, w.il, s)) return st;
+        if (int st = il_factor(H, n, (int)n, r, L, lambda_rel, w.Uaug, w.f.A, w.f.T, lambda_out,
+                               w.il, s))
+            return st;
+    }
+    if (int st = init_work(W, w_dtype, m, (int)n, w.q.Wc, N, (int)N, s)) return st;
+    if (int st = sweep_layer(w.q.Wc, N, (int)m, (int)n, (int)N, w.Uaug, N, bits, group_size,
+                             block_size, codes, scales, zeros, loss_out, w.q.Err, s))
+        return st;
+    if (r > 0) {
+        extract_R_kernel<<<592, 256, 0, s>>>(w.q.Wc, N, (int)m, (int)n, r, R);
+        return launch_status();
+    }
+    return GPTQ_OK;
+}
+
+}  // extern "C"

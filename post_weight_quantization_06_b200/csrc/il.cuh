@@ -1,0 +1,292 @@
+// GPTQ-intrinsic LoRA on the device.
+//
+// GPTQ-intrinsic LoRA summary, "Method" part 2: X~ = [X, X V_r] with V_r the top-r right
+// singular vectors of X; the pass runs on W~ = [W, 0]; the r extra coordinates absorb the
+// error and become R; the singular augmented Hessian is factored without a plain Cholesky.
+//
+// Device route:
+//   1. V_r: block subspace iteration on H (= 2 X^T X, same eigenvectors as X^T X) with
+//      CholeskyQR2 re-orthonormalisation, then a Rayleigh-Ritz step whose small p x p
+//      eigenproblem is solved by a one-CTA parallel-order Jacobi sweep.
+//   2. H~ = [[H + l I, H V], [V^T H, V^T H V + l I]] with l = lambda_rel * mean of
+//      its n + r raw diagonal entries. The first n rows of U~ (H~^-1 = U~^T U~) are
+//      [U11, U12] with U11 the factor of the Schur complement S = H + l I - H V C^-1 V^T H
+//      (C = V^T H V + l I) and U12 = -U11 H V C^-1. S is positive definite although H~ is
+//      singular up to l, so the plain blocked factor applies to it.
+//   3. The sweep on [W, 0] with those n rows; R = the final extra columns, transposed.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "factor.cuh"
+
+namespace gptq {
+
+constexpr int IL_MAX_R = 128;
+constexpr int IL_ITERS = 6;
+
+inline int il_block_p(int n, int r) {
+    int p = r + 32 > 2 * r ? r + 32 : 2 * r;
+    if (p > 128) p = 128;
+    if (p > n) p = n;
+    if (p & 1) p -= 1;
+    if (p < r) p = r;  // only when n == r (odd): p = r
+    return p;
+}
+
+__device__ __forceinline__ unsigned long long splitmix64(unsigned long long x) {
+    x += 0x9E3779B97F4A7C15ull;
+    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+    return x ^ (x >> 31);
+}
+
+// Deterministic start block: entries uniform in (-1, 1) from a counter hash.
+__global__ void random_block_kernel(float *Y, long long total, unsigned long long seed) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+         i += (long long)gridDim.x * blockDim.x) {
+        const unsigned long long h = splitmix64(seed ^ (unsigned long long)i * 0xD1B54A32D192ED03ull);
+        Y[i] = (float)((double)(h >> 11) * (2.0 / 9007199254740992.0) - 1.0);
+    }
+}
+
+// One-CTA cyclic Jacobi on a symmetric p x p matrix (p even, p <= 128), round-robin
+// ordering so that p/2 disjoint rotations run at once. On exit: eigenvalues on the
+// diagonal of T; eigenvectors in the columns of Q. Then the r largest are selected in
+// decreasing order: evals[0..r), Qsel (p x r, column c = eigenvector of the c-th largest).
+__global__ __launch_bounds__(512) void jacobi_eig_kernel(const float *Tin, int p, int r,
+                                                         float *Qsel, float *evals) {
+    extern __shared__ float sm[];
+    const int LD = p + 1;
+    float *T = sm;
+    float *Q = T + p * LD;
+    float *cs = Q + p * LD;       // p/2 cosines
+    float *sn = cs + p / 2;       // p/2 sines
+    int *pi = reinterpret_cast<int *>(sn + p / 2);
+    int *pj = pi + p / 2;
+    __shared__ float off_s;
+    const int tid = threadIdx.x, nt = blockDim.x;
+    for (int idx = tid; idx < p * p; idx += nt) {
+        const int i = idx / p, j = idx % p;
+        T[i * LD + j] = 0.5f * (Tin[i * p + j] + Tin[j * p + i]);
+        Q[i * LD + j] = (i == j) ? 1.f : 0.f;
+    }
+    __syncthreads();
+    const int half = p / 2;
+    for (int sweep = 0; sweep < 15; ++sweep) {
+        // off-diagonal mass relative to the diagonal
+        if (tid == 0) off_s = 0.f;
+        __syncthreads();
+        float loc = 0.f, dg = 0.f;
+        for (int idx = tid; idx < p * p; idx += nt) {
+            const int i = idx / p, j = idx % p;
+            const float v = T[i * LD + j];
+            if (i != j) loc += v * v; else dg += v * v;
+        }
+        atomicAdd(&off_s, loc);
+        __syncthreads();
+        const float off = off_s;
+        __syncthreads();
+        if (tid == 0) off_s = 0.f;
+        __syncthreads();
+        atomicAdd(&off_s, dg);
+        __syncthreads();
+        const float dia = off_s;
+        __syncthreads();
+        if (off <= 1e-10f * dia) break;
+        for (int rnd = 0; rnd < p - 1; ++rnd) {
+            for (int k = tid; k < half; k += nt) {
+                // circle method: position 0 fixed, positions 1..p-1 rotate
+                const int xa = k, xb = p - 1 - k;
+                const int a = xa == 0 ? 0 : 1 + (xa - 1 + rnd) % (p - 1);
+                const int b = 1 + (xb - 1 + rnd) % (p - 1);
+                const int i = min(a, b), j = max(a, b);
+                pi[k] = i; pj[k] = j;
+                const float aij = T[i * LD + j];
+                float c = 1.f, s = 0.f;
+                if (aij != 0.f) {
+                    const float tau = (T[j * LD + j] - T[i * LD + i]) / (2.f * aij);
+                    const float t = (tau >= 0.f ? 1.f : -1.f) / (fabsf(tau) + sqrtf(1.f + tau * tau));
+                    c = rsqrtf(1.f + t * t);
+                    s = t * c;
+                }
+                cs[k] = c; sn[k] = s;
+            }
+            __syncthreads();
+            // rows: row_i <- c row_i - s row_j ; row_j <- s row_i + c row_j
+            for (int idx = tid; idx < half * p; idx += nt) {
+                const int k = idx / p, l = idx % p;
+                const int i = pi[k], j = pj[k];
+                const float c = cs[k], s = sn[k];
+                const float ti = T[i * LD + l], tj = T[j * LD + l];
+                T[i * LD + l] = c * ti - s * tj;
+                T[j * LD + l] = s * ti + c * tj;
+            }
+            __syncthreads();
+            // columns of T and of Q
+            for (int idx = tid; idx < half * p; idx += nt) {
+                const int k = idx / p, l = idx % p;
+                const int i = pi[k], j = pj[k];
+                const float c = cs[k], s = sn[k];
+                const float ti = T[l * LD + i], tj = T[l * LD + j];
+                T[l * LD + i] = c * ti - s * tj;
+                T[l * LD + j] = s * ti + c * tj;
+                const float qi = Q[l * LD + i], qj = Q[l * LD + j];
+                Q[l * LD + i] = c * qi - s * qj;
+                Q[l * LD + j] = s * qi + c * qj;
+            }
+            __syncthreads();
+        }
+    }
+    // rank by decreasing eigenvalue (ties by index)
+    for (int i = tid; i < p; i += nt) {
+        const float li = T[i * LD + i];
+        int rank = 0;
+        for (int j = 0; j < p; ++j) {
+            const float lj = T[j * LD + j];
+            rank += (lj > li) || (lj == li && j < i);
+        }
+        if (rank < r) {
+            evals[rank] = li;
+            for (int l = 0; l < p; ++l) Qsel[l * r + rank] = Q[l * LD + i];
+        }
+    }
+}
+
+// Columns of V (n x r): flip so that the largest-magnitude entry (first on ties) is positive.
+__global__ void sign_fix_kernel(float *V, int n, int r) {
+    const int c = blockIdx.x;
+    __shared__ float bv[32];
+    __shared__ int bi[32];
+    float best = -1.f;
+    int besti = 0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const float a = fabsf(V[(long long)i * r + c]);
+        if (a > best) { best = a; besti = i; }
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, besti, o);
+        if (ob > best || (ob == best && oi < besti)) { best = ob; besti = oi; }
+    }
+    if ((threadIdx.x & 31) == 0) { bv[threadIdx.x >> 5] = best; bi[threadIdx.x >> 5] = besti; }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int w = 1; w < (int)(blockDim.x >> 5); ++w)
+            if (bv[w] > best || (bv[w] == best && bi[w] < besti)) { best = bv[w]; besti = bi[w]; }
+        bi[0] = besti;
+    }
+    __syncthreads();
+    const bool flip = V[(long long)bi[0] * r + c] < 0.f;
+    if (flip)
+        for (int i = threadIdx.x; i < n; i += blockDim.x) V[(long long)i * r + c] = -V[(long long)i * r + c];
+}
+
+// l~ = lambda_rel * (sum diag H + sum diag C) / (n + r); then C += l~ I.
+__global__ void il_lambda_kernel(const float *H, long long ldh, int n, float *C, int r,
+                                 float lambda_rel, float *lam) {
+    __shared__ double part[32];
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < n + r; i += blockDim.x) {
+        const float d = i < n ? H[(long long)i * ldh + i] : C[(i - n) * r + (i - n)];
+        if (i < n && !isfinite(d)) report(GPTQ_ERR_NONFINITE, (long long)i * ldh + i);
+        acc += d;
+    }
+    acc = warp_sum_d(acc);
+    if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = acc;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        double v = threadIdx.x < (blockDim.x >> 5) ? part[threadIdx.x] : 0.0;
+        v = warp_sum_d(v);
+        if (threadIdx.x == 0) part[0] = v;
+    }
+    __syncthreads();
+    const float l = (float)((double)lambda_rel * part[0] / (double)(n + r));
+    if (threadIdx.x == 0) *lam = l;
+    for (int i = threadIdx.x; i < r; i += blockDim.x) C[i * r + i] += l;
+}
+
+struct ILWork {
+    float *Y, *Z, *G, *Gi, *Tm, *Qsel, *ev;   // subspace iteration
+    float *B12, *C, *Ci, *Y1, *Yr;            // Schur pieces
+};
+
+inline int small_ul_inverse(float *M, float *Mi, int p, cudaStream_t s) {
+    // p <= FACTOR_NB: M = Ubar Ubar^T, Mi = Ubar^-1 (diag kernel; errors here are reported
+    // like any other non-positive pivot)
+    const int smem = 2 * FACTOR_NB * (FACTOR_NB + 1) * (int)sizeof(float);
+    cudaFuncSetAttribute(diag_ul_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    diag_ul_kernel<<<1, 512, smem, s>>>(M, p, Mi, p, 0, p);
+    return launch_status();
+}
+
+// Top-r eigenvectors of H (n x n) into V (n x r).
+inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V, ILWork &w,
+                          cudaStream_t s) {
+    const int p = il_block_p(n, r);
+    random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
+    GPTQ_CHECK_LAUNCH();
+    for (int it = 0; it < IL_ITERS; ++it) {
+        // Z = H Y
+        if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
+        // CholeskyQR2: Y = Z (Z^T Z)^-1/2-ish, twice
+        for (int pass = 0; pass < 2; ++pass) {
+            const float *src = pass == 0 ? w.Z : w.Y;
+            float *dst = pass == 0 ? w.Y : w.Z;
+            if (int st = gemm_simt(gemm_args<float, float>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.f, 0.f), s)) return st;
+            if (int st = small_ul_inverse(w.G, w.Gi, p, s)) return st;
+            // G = Ubar Ubar^T: src = (src Ubar^-T) Ubar^T, and src Ubar^-T has orthonormal columns
+            if (int st = gemm_simt(gemm_args<float, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.f, 0.f), s)) return st;
+        }
+        // the orthonormal block is now in Z; move it to Y
+        cudaMemcpyAsync(w.Y, w.Z, sizeof(float) * (size_t)n * p, cudaMemcpyDeviceToDevice, s);
+    }
+    // Rayleigh-Ritz: Tm = Y^T H Y
+    if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
+    if (int st = gemm_simt(gemm_args<float, float>(p, p, n, w.Y, p, 1, w.Z, p, 0, w.Tm, p, 1.f, 0.f), s)) return st;
+    const int smem = (2 * p * (p + 1) + 2 * p) * (int)sizeof(float);
+    cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    jacobi_eig_kernel<<<1, 512, smem, s>>>(w.Tm, p, r, w.Qsel, w.ev);
+    GPTQ_CHECK_LAUNCH();
+    // V = Y Qsel
+    if (int st = gemm_simt(gemm_args<float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.f, 0.f), s)) return st;
+    sign_fix_kernel<<<r, 256, 0, s>>>(V, n, r);
+    return launch_status();
+}
+
+// First n rows of U~ into Uaug (n x (n + r), ldu = n + r), lambda~ into *lam.
+// Awork: n x n scratch, T: FACTOR_NB x n scratch.
+inline int il_factor(const float *H, long long ldh, int n, int r, const float *V,
+                     float lambda_rel, float *Uaug, float *Awork, float *T, float *lam,
+                     ILWork &w, cudaStream_t s) {
+    const long long ldu = n + r;
+    // B12 = H V (n x r), C = V^T B12 (r x r)
+    if (int st = gemm_simt(gemm_args<float, float>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.f, 0.f), s)) return st;
+    if (int st = gemm_simt(gemm_args<float, float>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.f, 0.f), s)) return st;
+    il_lambda_kernel<<<1, 1024, 0, s>>>(H, ldh, n, w.C, r, lambda_rel, lam);
+    GPTQ_CHECK_LAUNCH();
+    // C = Ubar Ubar^T, Ci = Ubar^-1 ; C^-1 = Ci^T Ci
+    if (int st = small_ul_inverse(w.C, w.Ci, r, s)) return st;
+    // Y1 = B12 Ci^T (n x r);  S = H + l I - Y1 Y1^T ; Yr = Y1 Ci = B12 C^-1
+    if (int st = gemm_simt(gemm_args<float, float>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.f, 0.f), s)) return st;
+    {
+        auto p = gemm_args<float, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.f, 0.f);
+        p.b_upper = 1;
+        if (int st = gemm_simt(p, s)) return st;
+    }
+    copy_damped_kernel<<<1184, 256, 0, s>>>(H, ldh, Awork, n, n, lam);
+    GPTQ_CHECK_LAUNCH();
+    {
+        auto p = gemm_args<float, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.f, 1.f);
+        p.c_upper = 1;
+        if (int st = gemm_simt(p, s)) return st;
+    }
+    cudaMemsetAsync(Uaug, 0, sizeof(float) * (size_t)n * ldu, s);
+    if (int st = factor_ul_inverse(Awork, n, Uaug, ldu, n, T, s)) return st;
+    // U12 = -U11 Yr
+    auto p = gemm_args<float, float>(n, r, n, Uaug, ldu, 0, w.Yr, r, 0, Uaug + n, ldu, -1.f, 0.f);
+    p.a_upper = 1;
+    return gemm_simt(p, s);
+}
+
+}  // namespace gptq

@@ -1,0 +1,286 @@
+// The column sweep: per-group min-max grid, quantize/round/clamp, error feedback inside a
+// panel of B columns, and the lazy trailing update once per panel.
+//
+// GPTQ (encyclopedia article), "Technical approach": columns are quantized one at a time
+// and the remaining weights are corrected in closed form; groups carry their own scale.
+// GPTQ-2D, section 2: errors of a block are flushed to the rest of the matrix with one
+// matrix product (GPTQ's lazy block update).
+#pragma once
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+
+namespace gptq {
+
+// Wc[i, c] = W[i, c] for c < n, 0 for n <= c < N (the intrinsic-LoRA extra columns).
+template <typename TW>
+__global__ void init_work_kernel(const TW *W, long long m, int n, float *Wc, long long ldw, int N) {
+    const long long total = m * (long long)N;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long row = idx / N;
+        const int c = (int)(idx % N);
+        float v = 0.f;
+        if (c < n) {
+            v = to_f32(W[row * n + c]);
+            if (!isfinite(v)) report(GPTQ_ERR_NONFINITE, row * n + c);
+        }
+        Wc[row * ldw + c] = v;
+    }
+}
+
+struct ColloopArgs {
+    float *Wc;          // m x N working weights (row stride ldw)
+    long long ldw;
+    const float *U;     // n x N upper factor rows (row stride ldu)
+    long long ldu;
+    int m, n;           // rows, quantized columns
+    int j0;             // first column of this panel
+    int bits;
+    int gs;             // group length (n when there is one group per row)
+    uint32_t *codes;    // m x (n*bits/32)
+    long long ldcodes;
+    float *scales;      // m x G
+    uint8_t *zeros;     // m x G
+    int G;
+    float *err;         // m x B errors of this panel (row stride B)
+    double *loss;       // m or nullptr
+};
+
+// Grid of one group from its range: s = (xmax - xmin)/maxq, z = rint(-xmin/s) in [0, maxq].
+__device__ __forceinline__ void grid_from_range(float mn, float mx, float fmaxq, float &s,
+                                                float &is, float &z) {
+    mn = fminf(mn, 0.f);
+    mx = fmaxf(mx, 0.f);
+    if (mx == mn) { mn = -1.f; mx = 1.f; }
+    s = __fdiv_rn(mx - mn, fmaxq);
+    is = __frcp_rn(s);
+    z = fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.f), fmaxq);
+}
+
+// One CTA = 8 warps; one warp = ROWS rows; lane l owns columns l, l+32, ... of the panel.
+// The panel's U block (B x B) and 1/U_jj sit in shared memory. Per column t: the owner
+// lane's value is broadcast by shuffle, every lane evaluates the rounding of that column
+// for its rows (the same value on all lanes), and each lane applies -e * U[t, col] to the
+// columns it owns that come after t.
+template <int NSLOT, int ROWS>
+__global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
+    constexpr int B = 32 * NSLOT;
+    extern __shared__ float sm[];
+    float *Us = sm;
+    float *invd = Us + B * B;
+    uint8_t *cbuf = reinterpret_cast<uint8_t *>(invd + B);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = blockDim.x >> 5;
+    const int j0 = a.j0;
+    for (int idx = tid; idx < B * B; idx += blockDim.x) {
+        const int t = idx / B, c = idx % B;
+        Us[idx] = a.U[(long long)(j0 + t) * a.ldu + j0 + c];
+    }
+    __syncthreads();
+    for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
+    __syncthreads();
+
+    const int maxq = (1 << a.bits) - 1;
+    const float fmaxq = (float)maxq;
+    const int row0 = (blockIdx.x * nwarps + warp) * ROWS;
+    float w[ROWS][NSLOT], ev[ROWS][NSLOT];
+    int cv[ROWS][NSLOT];
+    float s[ROWS], is[ROWS], z[ROWS], lacc[ROWS];
+    bool rv[ROWS];
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        const int row = row0 + r;
+        rv[r] = row < a.m;
+        lacc[r] = 0.f;
+        s[r] = 1.f; is[r] = 1.f; z[r] = 0.f;
+#pragma unroll
+        for (int q = 0; q < NSLOT; ++q) {
+            w[r][q] = rv[r] ? a.Wc[(long long)row * a.ldw + j0 + 32 * q + lane] : 0.f;
+            ev[r][q] = 0.f;
+            cv[r][q] = 0;
+        }
+    }
+    const int gs = a.gs;
+    const bool groups_in_panel = gs <= B;  // then B % gs == 0
+    if (!groups_in_panel) {
+        const int g = j0 / gs;
+        if (j0 % gs == 0) {
+            const int cend = min(j0 + gs, a.n);
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const int row = row0 + r;
+                float mn = INFINITY, mx = -INFINITY;
+                if (rv[r])
+                    for (int c = j0 + lane; c < cend; c += 32) {
+                        const float x = a.Wc[(long long)row * a.ldw + c];
+                        mn = fminf(mn, x);
+                        mx = fmaxf(mx, x);
+                    }
+                mn = warp_min(mn);
+                mx = warp_max(mx);
+                grid_from_range(mn, mx, fmaxq, s[r], is[r], z[r]);
+                if (lane == 0 && rv[r]) {
+                    a.scales[(long long)row * a.G + g] = s[r];
+                    a.zeros[(long long)row * a.G + g] = (uint8_t)z[r];
+                }
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const int row = row0 + r;
+                if (rv[r]) {
+                    s[r] = a.scales[(long long)row * a.G + g];
+                    z[r] = (float)a.zeros[(long long)row * a.G + g];
+                    is[r] = __frcp_rn(s[r]);
+                }
+            }
+        }
+    }
+
+#pragma unroll
+    for (int q = 0; q < NSLOT; ++q) {
+#pragma unroll 2
+        for (int o = 0; o < 32; ++o) {
+            const int t = 32 * q + o;
+            if (groups_in_panel && (t % gs) == 0) {
+                const int g = (j0 + t) / gs;
+#pragma unroll
+                for (int r = 0; r < ROWS; ++r) {
+                    float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+                    for (int q2 = 0; q2 < NSLOT; ++q2) {
+                        const int col = 32 * q2 + lane;
+                        if (q2 >= q && col >= t && col < t + gs) {
+                            mn = fminf(mn, w[r][q2]);
+                            mx = fmaxf(mx, w[r][q2]);
+                        }
+                    }
+                    mn = warp_min(mn);
+                    mx = warp_max(mx);
+                    grid_from_range(mn, mx, fmaxq, s[r], is[r], z[r]);
+                    if (lane == 0 && rv[r]) {
+                        const int row = row0 + r;
+                        a.scales[(long long)row * a.G + g] = s[r];
+                        a.zeros[(long long)row * a.G + g] = (uint8_t)z[r];
+                    }
+                }
+            }
+            const float ut = invd[t];
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                const float wt = __shfl_sync(0xffffffffu, w[r][q], o);
+                const float v = fmaf(wt, is[r], z[r]);
+                const float c = fminf(fmaxf(rintf(v), 0.f), fmaxq);
+                const float wq = s[r] * (c - z[r]);
+                const float e = (wt - wq) * ut;
+                lacc[r] = fmaf(e, e, lacc[r]);
+                if (lane == o) {
+                    cv[r][q] = (int)c;
+                    ev[r][q] = e;
+                }
+#pragma unroll
+                for (int q2 = q; q2 < NSLOT; ++q2) {
+                    const int col = 32 * q2 + lane;
+                    if (q2 > q || lane > o) w[r][q2] = fmaf(-e, Us[t * B + col], w[r][q2]);
+                }
+            }
+        }
+    }
+
+    // errors of the panel (for the lazy update), loss, packed codes
+    uint8_t *cb = cbuf + warp * ROWS * B;
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        const int row = row0 + r;
+#pragma unroll
+        for (int q = 0; q < NSLOT; ++q) {
+            if (rv[r]) a.err[(long long)row * B + 32 * q + lane] = ev[r][q];
+            cb[r * B + 32 * q + lane] = (uint8_t)cv[r][q];
+        }
+        if (a.loss && lane == 0 && rv[r]) {
+            if (j0 == 0) a.loss[row] = (double)lacc[r];
+            else a.loss[row] += (double)lacc[r];
+        }
+    }
+    __syncwarp();
+    const int bits = a.bits;
+    const int wpp = B * bits / 32;  // words per row for this panel
+#pragma unroll
+    for (int r = 0; r < ROWS; ++r) {
+        const int row = row0 + r;
+        if (!rv[r] || lane >= wpp) continue;
+        const int bit0 = lane * 32;
+        const int cfirst = bit0 / bits, clast = min(B - 1, (bit0 + 31) / bits);
+        uint32_t word = 0;
+        for (int c = cfirst; c <= clast; ++c) {
+            const int pos = c * bits - bit0;
+            const uint32_t code = cb[r * B + c];
+            word |= pos >= 0 ? (code << pos) : (code >> (-pos));
+        }
+        a.codes[(long long)row * a.ldcodes + (long long)j0 * bits / 32 + lane] = word;
+    }
+}
+
+constexpr int COLLOOP_ROWS = 2;
+constexpr int COLLOOP_THREADS = 256;
+
+template <int NSLOT>
+inline size_t colloop_smem() {
+    constexpr int B = 32 * NSLOT;
+    return (size_t)B * B * 4 + B * 4 + (COLLOOP_THREADS / 32) * COLLOOP_ROWS * B;
+}
+
+template <int NSLOT>
+inline int colloop_launch(const ColloopArgs &a, cudaStream_t s) {
+    const size_t smem = colloop_smem<NSLOT>();
+    cudaFuncSetAttribute(colloop_kernel<NSLOT, COLLOOP_ROWS>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int rows_per_cta = (COLLOOP_THREADS / 32) * COLLOOP_ROWS;
+    colloop_kernel<NSLOT, COLLOOP_ROWS>
+        <<<ceil_div(a.m, rows_per_cta), COLLOOP_THREADS, smem, s>>>(a);
+    return launch_status();
+}
+
+// R[t, i] = Wc[i, n + t]: the extra columns, transposed to r x m.
+__global__ void extract_R_kernel(const float *Wc, long long ldw, int m, int n, int r, float *R) {
+    const long long total = (long long)r * m;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int t = (int)(idx / m), i = (int)(idx % m);
+        R[idx] = Wc[(long long)i * ldw + n + t];
+    }
+}
+
+// The sweep over all panels of a prepared working copy Wc (m x N, first n columns quantized).
+inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const float *U,
+                       long long ldu, int bits, int group_size, int B, uint32_t *codes,
+                       float *scales, uint8_t *zeros, double *loss, float *Err,
+                       cudaStream_t s) {
+    ColloopArgs a;
+    a.Wc = Wc; a.ldw = ldw; a.U = U; a.ldu = ldu; a.m = m; a.n = n;
+    a.bits = bits; a.gs = group_size ? group_size : n;
+    a.codes = codes; a.ldcodes = (long long)n * bits / 32;
+    a.scales = scales; a.zeros = zeros; a.G = group_size ? n / group_size : 1;
+    a.err = Err; a.loss = loss;
+    for (int j0 = 0; j0 < n; j0 += B) {
+        a.j0 = j0;
+        int st;
+        switch (B) {
+            case 32: st = colloop_launch<1>(a, s); break;
+            case 64: st = colloop_launch<2>(a, s); break;
+            default: st = colloop_launch<4>(a, s); break;
+        }
+        if (st) return st;
+        const int j1 = j0 + B;
+        if (j1 < N) {
+            // Wc[:, j1:N] -= Err (m x B) * U[j0:j1, j1:N]
+            auto p = gemm_args<float, float>(m, N - j1, B, Err, B, 0, U + (long long)j0 * ldu + j1,
+                                             ldu, 0, Wc + j1, ldw, -1.f, 1.f);
+            if (int st2 = gemm_simt(p, s)) return st2;
+        }
+    }
+    return GPTQ_OK;
+}
+
+}  // namespace gptq

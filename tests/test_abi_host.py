@@ -1,0 +1,130 @@
+"""Host-side checks of the C ABI: the library loads, exports what include/gptq.h declares,
+and rejects bad arguments before touching the device (no GPU needed)."""
+import ctypes
+import importlib
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "gptq.h")).read()
+    return sorted(set(re.findall(r"GPTQ_API\s+[\w\s\*]+?\b(gptq_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    assert _declared() == sorted([
+        "gptq_workspace_size", "gptq_status_string", "gptq_sync_status",
+        "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
+        "gptq_il_quantize_layer"])
+
+
+def test_library_exports_every_declared_symbol():
+    import post_weight_quantization_06_b200 as g
+    out = subprocess.run(["nm", "-D", "--defined-only", g.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, re.M))
+    for name in _declared():
+        assert name in exported, name
+    lib = ctypes.CDLL(g.LIB_PATH)
+    for name in _declared():
+        assert getattr(lib, name) is not None
+    assert set(g.EXPORTED) == set(_declared())
+
+
+def test_library_has_no_dynamic_cuda_runtime_dependency():
+    import post_weight_quantization_06_b200 as g
+    out = subprocess.run(["ldd", g.LIB_PATH], capture_output=True, text=True).stdout
+    assert "libcudart" not in out
+
+
+def test_status_strings():
+    import post_weight_quantization_06_b200 as g
+    assert g.status_string(0) == "GPTQ_OK"
+    for code in range(-6, 0):
+        assert g.status_string(code).startswith("GPTQ_ERR_")
+    assert "unknown" in g.status_string(7)
+
+
+def test_workspace_sizes():
+    import post_weight_quantization_06_b200 as g
+    assert g.gptq_workspace_size(g.GPTQ_OP_HESSIAN, 10, 64) == 0
+    f = g.gptq_workspace_size(g.GPTQ_OP_PREPARE_HINV, 0, 6144)
+    assert f >= 6144 * 6144 * 4
+    q = g.gptq_workspace_size(g.GPTQ_OP_QUANTIZE, 2048, 6144, 0, 128)
+    assert q >= 2048 * 6144 * 4 + 2048 * 128 * 4
+    il0 = g.gptq_workspace_size(g.GPTQ_OP_IL_QUANTIZE, 2048, 6144, 0, 128)
+    il = g.gptq_workspace_size(g.GPTQ_OP_IL_QUANTIZE, 2048, 6144, 64, 128)
+    assert il > il0 >= q + f
+    assert g.gptq_workspace_size(99, 1, 1) == 0
+    for v in (f, q, il0, il):
+        assert v % 256 == 0
+
+
+def _lib():
+    import post_weight_quantization_06_b200 as g
+    return g._lib
+
+
+NULL = None
+P = ctypes.c_void_p(256)  # never dereferenced: every case below fails validation first
+
+
+@pytest.mark.parametrize("args", [
+    (NULL, P, 0, 10, 64, NULL),      # H missing
+    (P, P, 5, 10, 64, NULL),         # bad dtype
+    (P, P, 0, -1, 64, NULL),         # negative k
+    (P, P, 0, 10, 0, NULL),          # n = 0
+])
+def test_hessian_rejects_bad_arguments(args):
+    assert _lib().gptq_hessian_accumulate(*args) == -1
+
+
+def test_hessian_k0_is_a_noop():
+    assert _lib().gptq_hessian_accumulate(P, P, 0, 0, 64, NULL) == 0
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(bits=1), -1), (dict(bits=9), -1), (dict(block=96), -1), (dict(n=200), -1),
+    (dict(gs=48), -1), (dict(gs=100, n=1000, block=100), -1), (dict(m=0), -1),
+    (dict(ws_bytes=16), -6), (dict(ws=None), -6),
+])
+def test_quantize_rejects_bad_arguments(kw, expect):
+    import post_weight_quantization_06_b200 as g
+    a = dict(m=64, n=256, bits=4, gs=128, block=128, ws=ctypes.c_void_p(1 << 20), ws_bytes=None)
+    a.update(kw)
+    ws_bytes = a["ws_bytes"]
+    if ws_bytes is None:
+        ws_bytes = g.gptq_workspace_size(g.GPTQ_OP_QUANTIZE, max(a["m"], 1), a["n"], 0, a["block"])
+    st = _lib().gptq_quantize_layer(P, 1, a["m"], a["n"], P, a["bits"], a["gs"], a["block"],
+                                    P, P, P, NULL, a["ws"], ws_bytes, NULL)
+    assert st == expect
+
+
+def test_workspace_alignment_is_checked():
+    import post_weight_quantization_06_b200 as g
+    need = g.gptq_workspace_size(g.GPTQ_OP_PREPARE_HINV, 0, 64)
+    st = _lib().gptq_prepare_hinv(P, 64, ctypes.c_float(0.01), P, P, ctypes.c_void_p((1 << 20) + 64),
+                                  need, NULL)
+    assert st == -6
+
+
+@pytest.mark.parametrize("r,L,lam", [(-1, P, 0.01), (129, P, 0.01), (4, NULL, 0.01), (256, P, 0.01),
+                                     (4, P, -1.0), (4, P, float("nan"))])
+def test_il_rejects_bad_arguments(r, L, lam):
+    import post_weight_quantization_06_b200 as g
+    need = g.gptq_workspace_size(g.GPTQ_OP_IL_QUANTIZE, 64, 256, max(r, 0), 128)
+    st = _lib().gptq_il_quantize_layer(P, 1, 64, 256, P, r, 4, 128, ctypes.c_float(lam), 128,
+                                       P, P, P, L, P, P, NULL, ctypes.c_void_p(1 << 20), need, NULL)
+    assert st == -1
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    import post_weight_quantization_06_b200 as g
+    monkeypatch.setattr(g, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(ImportError):
+        g._load()

@@ -1,0 +1,448 @@
+#!/usr/bin/env python
+"""Benchmark of the GPTQ layer pass on B200: ms per layer and weights quantized per second.
+
+One step = the whole pass over one layer, through the C ABI:
+    H = 0; gptq_hessian_accumulate over all calibration tokens (2 X^T X)
+    gptq_prepare_hinv (damping + factor U)      | or gptq_il_quantize_layer
+    gptq_quantize_layer (sweep, lazy updates)   |    (intrinsic-LoRA workload)
+Default workload: the 2048 x 6144 MLP down-projection layer, 262144 bf16 calibration tokens,
+3-bit, groups of 128, lambda = 0.01 mean(diag H), B = 128 (synthetic data).
+
+Timing: W untimed warm-up steps, then K steps between a barrier + device synchronize on each
+side, timed with CUDA events on the launching stream; the calibration set (3.2 GB) is larger
+than L2, so no flush is needed. With --gpus N (torchrun), each rank quantizes its own layer
+(independent problems, no data-path collective): weak scaling, max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the same
+workload and extrapolates to the same metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "weights quantized per second (GPTQ layer pass, 1 layer per GPU per step)"
+UNIT = "weights/s"
+WORKLOAD_SEEDS = {"tiny": 0, "attn": 1, "mlp_down": 2, "deit_fc1": 3, "deit_fc2": 3, "lowrank": 4}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mlp_down", choices=sorted(WORKLOAD_SEEDS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------------------------------
+# ranks
+# ------------------------------------------------------------------------------------------
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Rank 0 quantizes the workload's own seeded layer; rank r > 0 an independent layer of
+    the same recipe (weak scaling: one layer per GPU per step)."""
+    return WORKLOAD_SEEDS[workload] + 1000 * rank
+
+
+def reduce_max(value: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = [ln.split(",") for ln in open(self.path).read().strip().splitlines() if ln.strip()]
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if len(r) >= 9 and r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if len(r) >= 9 and r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            if len(r) < 9:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------------------------------
+# device arm
+# ------------------------------------------------------------------------------------------
+
+class LayerPass:
+    """Buffers and calls of one layer pass through the C ABI."""
+
+    def __init__(self, g, layer, stream):
+        self.g, self.L, self.s = g, layer, stream
+        dev = layer.W.device
+        m, n, r = layer.m, layer.n, layer.r
+        G = n // layer.group_size if layer.group_size else 1
+        self.H = torch.empty(n, n, dtype=torch.float32, device=dev)
+        self.U = torch.empty(n, n, dtype=torch.float32, device=dev)
+        self.codes = torch.empty(m, n * layer.bits // 32, dtype=torch.int32, device=dev)
+        self.scales = torch.empty(m, G, dtype=torch.float32, device=dev)
+        self.zeros = torch.empty(m, G, dtype=torch.uint8, device=dev)
+        self.loss = torch.empty(m, dtype=torch.float64, device=dev)
+        self.lam = torch.empty(1, dtype=torch.float32, device=dev)
+        if r:
+            self.Lr = torch.empty(n, r, dtype=torch.float32, device=dev)
+            self.R = torch.empty(r, m, dtype=torch.float32, device=dev)
+            self.ws = g.workspace(g.GPTQ_OP_IL_QUANTIZE, m, n, r, layer.block_size, dev)
+        else:
+            self.ws_f = g.workspace(g.GPTQ_OP_PREPARE_HINV, m, n, 0, layer.block_size, dev)
+            self.ws = g.workspace(g.GPTQ_OP_QUANTIZE, m, n, 0, layer.block_size, dev)
+        self.ev = self.new_events()
+
+    @staticmethod
+    def new_events():
+        return [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def hessian(self, X_chunks):
+        for X in X_chunks:
+            self.g.gptq_hessian_accumulate(self.H, X, stream=self.s)
+
+    def rest(self, W):
+        g, L, s = self.g, self.L, self.s
+        if L.r:
+            g.gptq_il_quantize_layer(W, self.H, L.r, L.bits, L.group_size, L.lambda_rel,
+                                     L.block_size, self.codes, self.scales, self.zeros, self.Lr,
+                                     self.R, self.lam, self.loss, self.ws, stream=s)
+        else:
+            g.gptq_prepare_hinv(self.H, L.lambda_rel, self.U, self.lam, self.ws_f, stream=s)
+            g.gptq_quantize_layer(W, self.U, L.bits, L.group_size, L.block_size, self.codes,
+                                  self.scales, self.zeros, self.loss, self.ws, stream=s)
+
+    def step(self, ev=None):
+        """Device-resident step with stage events: [start, H done, factor done, end]."""
+        if ev is not None:
+            self.ev = ev
+        with torch.cuda.stream(self.s):
+            self.ev[0].record(self.s)
+            self.H.zero_()
+            self.hessian([self.L.X])
+            self.ev[1].record(self.s)
+            if self.L.r:
+                self.ev[2].record(self.s)
+                self.rest(self.L.W)
+            else:
+                g, L = self.g, self.L
+                g.gptq_prepare_hinv(self.H, L.lambda_rel, self.U, self.lam, self.ws_f, stream=self.s)
+                self.ev[2].record(self.s)
+                g.gptq_quantize_layer(L.W, self.U, L.bits, L.group_size, L.block_size, self.codes,
+                                      self.scales, self.zeros, self.loss, self.ws, stream=self.s)
+            self.ev[3].record(self.s)
+
+    def stage_ms(self):
+        e = self.ev
+        return (e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
+
+    def outputs(self):
+        outs = [self.codes, self.scales, self.zeros, self.loss]
+        if self.L.r:
+            outs += [self.Lr, self.R]
+        return outs
+
+
+def hessian_flops(layer) -> float:
+    """Algorithmic flops of the Hessian: k n (n + 1) (one symmetric triangle)."""
+    return float(layer.k) * layer.n * (layer.n + 1)
+
+
+def run_e2e(g, layer, lp, steps, warmup, chunk_tokens=32768):
+    """Same pass, inputs from pinned host memory: per step the calibration chunks and W are
+    copied host -> device (copies of chunk i+1 overlap the Hessian of chunk i on a second
+    stream) and the packed codes, scales, zeros and loss are read back."""
+    dev = layer.W.device
+    X_host = layer.X.cpu().pin_memory()
+    W_host = layer.W.cpu().pin_memory()
+    k, n = layer.X.shape
+    bufs = [torch.empty(chunk_tokens, n, dtype=layer.X.dtype, device=dev) for _ in range(2)]
+    W_dev = torch.empty_like(layer.W)
+    outs_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in lp.outputs()]
+    cstream = torch.cuda.Stream(device=dev)
+    s = lp.s
+    copied = [torch.cuda.Event() for _ in range(2)]
+    used = [torch.cuda.Event() for _ in range(2)]
+    h2d = X_host.numel() * X_host.element_size() + W_host.numel() * W_host.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in outs_host)
+
+    def one():
+        with torch.cuda.stream(s):
+            lp.H.zero_()
+            for i, t0 in enumerate(range(0, k, chunk_tokens)):
+                t1 = min(k, t0 + chunk_tokens)
+                b = i % 2
+                cstream.wait_event(used[b]) if i >= 2 else cstream.wait_stream(s)
+                with torch.cuda.stream(cstream):
+                    bufs[b][: t1 - t0].copy_(X_host[t0:t1], non_blocking=True)
+                    copied[b].record(cstream)
+                s.wait_event(copied[b])
+                g.gptq_hessian_accumulate(lp.H, bufs[b][: t1 - t0], stream=s)
+                used[b].record(s)
+            W_dev.copy_(W_host, non_blocking=True)
+            lp.rest(W_dev)
+            for oh, od in zip(outs_host, lp.outputs()):
+                oh.copy_(od, non_blocking=True)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for _ in range(steps):
+        one()
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    ms = reduce_max(ms, dev)
+    barrier()
+    return ms, h2d, d2h
+
+
+def cpu_baseline(layer, budget_s: float):
+    """The fp64 oracle as it stands, on a bounded sample of the same layer, on the host cores:
+    Hessian over a slice of the tokens, the full n x n factor, the sweep over a few rows;
+    extrapolated linearly in tokens and rows to one whole layer."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max(int(i.get("num_threads", 1)) for i in threadpool_info()) if threadpool_info() else os.cpu_count()
+    except Exception:
+        cores = os.cpu_count()
+    k, n = layer.X.shape
+    m = layer.m
+    k_s = min(k, 4096)
+    m_s = min(m, 8)
+    X = layer.X[:k_s].double().cpu().numpy()
+    W = layer.W[:m_s].double().cpu().numpy()
+    t0 = time.perf_counter()
+    H = oracle.hessian(X)
+    t_h = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    if layer.r:
+        G = H / 2
+        V, _ = oracle.top_singular_directions(G, layer.r)
+        Ht, _ = oracle.il_hessian(G, V, layer.lambda_rel)
+        U = oracle.eig_qr_factor(Ht)[:n]
+        Wt = np.hstack([W, np.zeros((m_s, layer.r))])
+    else:
+        Hd, _ = oracle.damp(H, layer.lambda_rel)
+        U = oracle.inverse_cholesky_upper(Hd)
+        Wt = W
+    t_f = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.sweep(Wt, U, layer.bits, layer.group_size, n_quant=n)
+    t_s = time.perf_counter() - t0
+    total = t_h * (k / k_s) + t_f + t_s * (m / m_s)
+    return {
+        "value": m * n / total,
+        "unit": UNIT,
+        "cores": cores,
+        "kind": "oracle",
+        "seconds_per_layer": total,
+        "sample": (f"fp64 NumPy oracle: Hessian on {k_s} of {k} tokens ({t_h:.2f} s, scaled x{k / k_s:.0f}), "
+                   f"full {n}x{n} factor ({t_f:.2f} s), sweep of {m_s} of {m} rows "
+                   f"({t_s:.2f} s, scaled x{m / m_s:.0f}); {total:.0f} s per layer"),
+    }
+
+
+def bench_ours(args):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    import datagen
+    import post_weight_quantization_06_b200 as g
+
+    layer = datagen.WORKLOADS[args.workload](device=dev, seed=rank_seed(args.workload, rank))
+    stream = torch.cuda.Stream(device=dev)
+    lp = LayerPass(g, layer, stream)
+    for _ in range(args.warmup):
+        lp.step()
+    torch.cuda.synchronize(dev)
+    g.gptq_sync_status(stream)
+    barrier()
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    events = [LayerPass.new_events() for _ in range(args.steps)]
+    l0 = g.gptq_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0.record(stream)
+    for i in range(args.steps):
+        lp.step(events[i])
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = g.gptq_launch_count() - l0
+    stage = np.zeros(3)
+    for ev in events:
+        lp.ev = ev
+        stage += np.array(lp.stage_ms())
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = reduce_max(ms, dev)
+    barrier()
+    clk = clocks.stop()
+    st, info = g.gptq_sync_status(stream, raise_on_error=False)
+    stage /= args.steps
+
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else None
+    if peaks:
+        peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (bf16 sustained)"
+    else:
+        peak, peak_src = 1400.0, "fallback (bf16 sustained)"
+    h_tflops = hessian_flops(layer) / (stage[0] * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = run_e2e(g, layer, lp, max(1, min(args.steps, 3)), 1)
+        e2e = {"value": world * layer.m * layer.n / (e_ms * 1e-3), "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC,
+            "value": world * layer.m * layer.n / (ms * 1e-3),
+            "unit": UNIT,
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16 X / fp32 accumulate; fp32 factor and sweep",
+            "data": "synthetic (seeded; shapes and spectra of the named layer)",
+            "config": {"workload": layer.name, "m": layer.m, "n": layer.n, "k_tokens": layer.k,
+                       "bits": layer.bits, "group_size": layer.group_size, "r": layer.r,
+                       "block_size": layer.block_size, "lambda_rel": layer.lambda_rel,
+                       "l2": "inputs larger than L2 (X is %.1f GB)" % (layer.X.numel() * 2 / 1e9),
+                       "parallelism": f"{world} independent layers (one per GPU)"},
+            "stages_ms": {"hessian": stage[0], "factor": stage[1], "sweep": stage[2]},
+            "roofline": {"bound": "tensor", "kernel": "hessian (2 X^T X)",
+                         "achieved": h_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": h_tflops / peak, "peak_source": peak_src,
+                         "traffic": None},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+            "device_status": int(st),
+        }
+        if e2e:
+            out["e2e"] = e2e
+        if not args.no_cpu_baseline and world == 1:
+            out["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def bench_reference(args):
+    """The oracle on the host cores, each step a bounded sample of the workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import datagen
+    layer = datagen.WORKLOADS[args.workload](device="cuda" if torch.cuda.is_available() else "cpu",
+                                              seed=rank_seed(args.workload, 0))
+    for _ in range(args.warmup):
+        cpu_baseline(layer, args.cpu_budget_s)
+    vals, secs = [], []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cb = cpu_baseline(layer, args.cpu_budget_s)
+        vals.append(cb["value"])
+        secs.append(cb["seconds_per_layer"])
+    wall = time.perf_counter() - t0
+    value = float(np.median(vals))
+    print(json.dumps({
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": float(np.median(secs)) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; same layer as the device arm)",
+        "config": {"workload": layer.name, "m": layer.m, "n": layer.n, "k_tokens": layer.k},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
+                         "sample": cb["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": wall,
+    }))
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        bench_reference(args)
+    else:
+        bench_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -77,6 +77,11 @@ GPTQ_API const char *gptq_status_string(int status);
  * NULL it receives the error's detail (column / index / site; 0 if none). */
 GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info);
 
+/* Number of CUDA kernels this library has launched in this process so far (all devices).
+ * A diagnostic for tracing and benchmarking: the difference of two readings counts the
+ * kernels a span of calls launched. Library-internal memsets are not counted. */
+GPTQ_API uint64_t gptq_launch_count(void);
+
 /*
  * H += 2 X^T X.
  * GPTQ (encyclopedia article), "Technical approach": the quantizer is driven by the

@@ -20,7 +20,7 @@ GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
 
-EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status",
+EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
             "gptq_il_quantize_layer")
 
@@ -41,6 +41,7 @@ def _load() -> ctypes.CDLL:
         "gptq_workspace_size": (c_sz, [c_int, c_i64, c_i64, c_int, c_int]),
         "gptq_status_string": (ctypes.c_char_p, [c_int]),
         "gptq_sync_status": (c_int, [c_p, ctypes.POINTER(c_i64)]),
+        "gptq_launch_count": (ctypes.c_uint64, []),
         "gptq_hessian_accumulate": (c_int, [c_p, c_p, c_int, c_i64, c_i64, c_p]),
         "gptq_prepare_hinv": (c_int, [c_p, c_i64, c_f, c_p, c_p, c_p, c_sz, c_p]),
         "gptq_quantize_layer": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int,
@@ -101,6 +102,11 @@ def workspace(op: int, m: int, n: int, r: int = 0, block_size: int = 128, device
     """A caller-owned workspace tensor (uint8, 256-byte aligned by the caching allocator)."""
     nbytes = gptq_workspace_size(op, m, n, r, block_size)
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def gptq_launch_count() -> int:
+    """Kernels launched by libgptq in this process so far."""
+    return int(_lib.gptq_launch_count())
 
 
 def gptq_sync_status(stream=None, raise_on_error: bool = True):

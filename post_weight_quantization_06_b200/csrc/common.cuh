@@ -6,6 +6,8 @@
 #include <stdint.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "gptq.h"
 
 namespace gptq {
@@ -55,7 +57,15 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
+// Every kernel launch of the library is followed by launch_status(), which also counts it
+// (read with gptq_launch_count()).
+inline std::atomic<unsigned long long> &launch_counter() {
+    static std::atomic<unsigned long long> c{0};
+    return c;
+}
+
 inline int launch_status() {
+    launch_counter().fetch_add(1, std::memory_order_relaxed);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

@@ -10,6 +10,7 @@
 //
 // Blocked, bottom-right first, with blocks of NB columns. For block p (rows r0..r1):
 //   1. diag:  A_pp = Ubar_pp Ubar_pp^T  and  U_pp = Ubar_pp^-1          (one CTA)
+//      (Ubar_pp itself is used by no later step)
 //   2. panel: Ubar[0:r0, p] = A[0:r0, p] U_pp^T                           (GEMM)
 //   3. syrk:  A[0:r0, 0:r0] -= Ubar[0:r0, p] Ubar[0:r0, p]^T (upper)       (GEMM)
 //   4. row p of U:  U[p, r1:] = -U_pp (Ubar[p, r1:] U[r1:, r1:])          (two GEMMs)
@@ -24,58 +25,71 @@ namespace gptq {
 
 constexpr int FACTOR_NB = 128;
 
-// One CTA: UL-Cholesky of the nb x nb diagonal block at A + r0*(lda+1) (upper triangle
-// read), and the inverse of its factor. Writes Ubar_pp to A's block (upper triangle) and
-// U_pp = Ubar_pp^-1 to U's block (upper; strictly lower part zeroed).
-// A pivot <= 0 (or NaN) records GPTQ_ERR_NOT_PD with the global column and continues with
-// a unit pivot so that the kernel always finishes.
-__global__ __launch_bounds__(512) void diag_ul_kernel(float *A, long long lda, float *U,
-                                                      long long ldu, int r0, int nb) {
-    extern __shared__ float sm[];
-    constexpr int LD = FACTOR_NB + 1;
-    float *S = sm;             // Ubar in progress, S[i*LD + j]
-    float *X = sm + FACTOR_NB * LD;  // inverse rows
+// One CTA: UL-Cholesky of an nb x nb symmetric block (upper triangle read) followed by the
+// inverse of its factor, in place in shared memory. On exit U's block holds
+// U_pp = Ubar_pp^-1 (upper; strictly lower part zeroed), where A_pp = Ubar_pp Ubar_pp^T.
+// Ubar_pp itself is not needed by any later step and is not stored.
+// Column c is processed from the last to the first: pivot, scaled column above it, update
+// of the leading block; then row c of the inverse, which only needs Ubar's row c (saved
+// first) and the rows of the inverse below it (already in place).
+// A pivot <= 0 (or NaN) records GPTQ_ERR_NOT_PD with info = col_base + c and continues with a
+// unit pivot so that the kernel always finishes.
+template <typename T>
+__global__ __launch_bounds__(512) void diag_ul_inv_kernel(const T *A, long long lda, T *U,
+                                                          long long ldu, int nb,
+                                                          long long col_base) {
+    extern __shared__ __align__(16) unsigned char smraw[];
+    T *S = reinterpret_cast<T *>(smraw);
+    T *rowc = S + nb * (nb + 1);
+    const int LD = nb + 1;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    float *Ab = A + (long long)r0 * lda + r0;
-    float *Ub = U + (long long)r0 * ldu + r0;
     for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
         const int i = idx / nb, j = idx % nb;
-        S[i * LD + j] = (j >= i) ? Ab[(long long)i * lda + j] : 0.f;
-        X[i * LD + j] = 0.f;
+        S[i * LD + j] = (j >= i) ? A[(long long)i * lda + j] : T(0);
     }
     __syncthreads();
     for (int c = nb - 1; c >= 0; --c) {
-        // pivot and scaled column c (above the diagonal)
-        float d = S[c * LD + c];
-        const bool bad = !(d > 0.f) || !isfinite(d);
-        if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, r0 + c);
-        const float piv = bad ? 1.f : sqrtf(d);
+        const T d = S[c * LD + c];
+        const bool bad = !(d > T(0)) || !isfinite((double)d);
+        if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
+        const T piv = bad ? T(1) : sqrt(d);
         __syncthreads();
         for (int i = tid; i < c; i += blockDim.x) S[i * LD + c] = S[i * LD + c] / piv;
-        if (tid == 0) S[c * LD + c] = piv;
+        for (int k = c + 1 + tid; k < nb; k += blockDim.x) rowc[k] = S[c * LD + k];
         __syncthreads();
-        // trailing update of the top-left block (upper triangle, rows/cols < c)
         for (int i = warp; i < c; i += nw) {
-            const float sic = S[i * LD + c];
+            const T sic = S[i * LD + c];
             for (int j = i + lane; j < c; j += 32) S[i * LD + j] -= sic * S[j * LD + c];
         }
-        // row c of the inverse: X[c][c] = 1/piv, X[c][j] = -X[c][c] * sum_{k=c+1..j} S[c][k] X[k][j]
-        const float xcc = 1.f / piv;
+        const T xcc = T(1) / piv;
         for (int j = c + 1 + warp; j < nb; j += nw) {
-            float acc = 0.f;
-            for (int k = c + 1 + lane; k <= j; k += 32) acc = fmaf(S[c * LD + k], X[k * LD + j], acc);
+            T acc = T(0);
+            for (int k = c + 1 + lane; k <= j; k += 32) acc += rowc[k] * S[k * LD + j];
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) X[c * LD + j] = -xcc * acc;
+            if (lane == 0) S[c * LD + j] = -xcc * acc;
         }
-        if (tid == 0) X[c * LD + c] = xcc;
+        if (tid == 0) S[c * LD + c] = xcc;
         __syncthreads();
     }
     for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
         const int i = idx / nb, j = idx % nb;
-        if (j >= i) Ab[(long long)i * lda + j] = S[i * LD + j];
-        Ub[(long long)i * ldu + j] = (j >= i) ? X[i * LD + j] : 0.f;
+        U[(long long)i * ldu + j] = (j >= i) ? S[i * LD + j] : T(0);
     }
+}
+
+template <typename T>
+inline size_t diag_smem(int nb) { return ((size_t)nb * (nb + 1) + nb) * sizeof(T); }
+
+// U_pp = inverse of the UL factor of the nb x nb block at A (nb <= FACTOR_NB).
+template <typename T>
+inline int diag_ul_inv(const T *A, long long lda, T *U, long long ldu, int nb, long long col_base,
+                       cudaStream_t s) {
+    const size_t smem = diag_smem<T>(FACTOR_NB);
+    cudaFuncSetAttribute(diag_ul_inv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    diag_ul_inv_kernel<T><<<1, 512, diag_smem<T>(nb), s>>>(A, lda, U, ldu, nb, col_base);
+    return launch_status();
 }
 
 // A_work = H + lambda I (full copy), lambda = lambda_rel * mean(diag H) written to *lam.
@@ -116,15 +130,14 @@ __global__ void copy_damped_kernel(const float *H, long long ldh, float *A, long
 // factor (upper; strictly lower part zero). T is scratch of FACTOR_NB x n floats.
 inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n,
                              float *T, cudaStream_t s) {
-    const int smem = 2 * FACTOR_NB * (FACTOR_NB + 1) * (int)sizeof(float);
-    cudaFuncSetAttribute(diag_ul_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     const int P = ceil_div(n, FACTOR_NB);
     for (int p = P - 1; p >= 0; --p) {
         const int r0 = p * FACTOR_NB;
         const int r1 = min(n, r0 + FACTOR_NB);
         const int nb = r1 - r0;
-        diag_ul_kernel<<<1, 512, smem, s>>>(A, lda, U, ldu, r0, nb);
-        GPTQ_CHECK_LAUNCH();
+        if (int st = diag_ul_inv<float>(A + (long long)r0 * lda + r0, lda,
+                                        U + (long long)r0 * ldu + r0, ldu, nb, r0, s))
+            return st;
         if (r0 > 0) {
             // 2. panel: A[0:r0, r0:r1] = A[0:r0, r0:r1] * U_pp^T  (in place: one column tile)
             auto pa = gemm_args<float, float>(r0, nb, nb, A + r0, lda, 0,

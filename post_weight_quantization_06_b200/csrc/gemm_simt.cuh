@@ -123,6 +123,80 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     return p;
 }
 
+template <typename T> __device__ __forceinline__ double to_f64(T x) { return (double)x; }
+template <> __device__ __forceinline__ double to_f64<__nv_bfloat16>(__nv_bfloat16 x) {
+    return (double)__bfloat162float(x);
+}
+
+// C = alpha * op(A) op(B) accumulated in fp64 (64 x 64 tiles, 4 x 4 per thread). For the
+// small and skinny products of the orthonormalisation steps, where fp32 accumulation would
+// lose the weak directions of an ill-conditioned block.
+template <typename TA, typename TB, typename TC>
+__global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, const TA *A,
+                                                          long long lda, int ta, const TB *B,
+                                                          long long ldb, int tb, TC *C,
+                                                          long long ldc, double alpha,
+                                                          int b_upper) {
+    constexpr int T = 64, BK = 16;
+    __shared__ double As[BK][T + 1];
+    __shared__ double Bs[BK][T + 1];
+    const int i0 = blockIdx.y * T, j0 = blockIdx.x * T;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    double acc[4][4] = {};
+    int kend = K;
+    if (b_upper) kend = min(kend, j0 + T);
+    for (int k0 = 0; k0 < kend; k0 += BK) {
+        for (int idx = tid; idx < T * BK; idx += 256) {
+            int r, kk;
+            if (ta) { kk = idx / T; r = idx % T; } else { r = idx / BK; kk = idx % BK; }
+            const int gi = i0 + r, gk = k0 + kk;
+            As[kk][r] = (gi < M && gk < kend)
+                            ? to_f64(ta ? A[(long long)gk * lda + gi] : A[(long long)gi * lda + gk])
+                            : 0.0;
+            int c;
+            if (tb) { c = idx / BK; kk = idx % BK; } else { kk = idx / T; c = idx % T; }
+            const int gj = j0 + c;
+            const int gk2 = k0 + kk;
+            Bs[kk][c] = (gj < N && gk2 < kend && (!b_upper || gk2 <= gj))
+                            ? to_f64(tb ? B[(long long)gj * ldb + gk2] : B[(long long)gk2 * ldb + gj])
+                            : 0.0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int kk = 0; kk < BK; ++kk) {
+            double a[4], b[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) { a[u] = As[kk][ty + 16 * u]; b[u] = Bs[kk][tx + 16 * u]; }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], b[v], acc[u][v]);
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int gi = i0 + ty + 16 * u;
+        if (gi >= M) continue;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const int gj = j0 + tx + 16 * v;
+            if (gj < N) C[(long long)gi * ldc + gj] = (TC)(alpha * acc[u][v]);
+        }
+    }
+}
+
+template <typename TA, typename TB, typename TC>
+inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, const TB *B,
+                       long long ldb, int tb, TC *C, long long ldc, double alpha, cudaStream_t s,
+                       int b_upper = 0) {
+    if (M <= 0 || N <= 0) return GPTQ_OK;
+    dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
+    gemm_f64acc_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, lda, ta, B, ldb, tb, C, ldc,
+                                                        alpha, b_upper);
+    return launch_status();
+}
+
 // Copy the upper triangle of an n x n matrix onto its lower triangle (32x32 smem tiles).
 __global__ void mirror_upper_kernel(float *H, long long ld, int n) {
     __shared__ float t[32][33];

@@ -62,16 +62,16 @@ inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
         const int p = il_block_p((int)n, r);
         w.il.Y = c.take<float>((size_t)n * p);
         w.il.Z = c.take<float>((size_t)n * p);
-        w.il.G = c.take<float>((size_t)p * p);
-        w.il.Gi = c.take<float>((size_t)p * p);
         w.il.Tm = c.take<float>((size_t)p * p);
         w.il.Qsel = c.take<float>((size_t)p * r);
         w.il.ev = c.take<float>((size_t)p);
+        w.il.G = c.take<double>((size_t)p * p);
+        w.il.Gi = c.take<double>((size_t)p * p);
         w.il.B12 = c.take<float>((size_t)n * r);
-        w.il.C = c.take<float>((size_t)r * r);
-        w.il.Ci = c.take<float>((size_t)r * r);
         w.il.Y1 = c.take<float>((size_t)n * r);
         w.il.Yr = c.take<float>((size_t)n * r);
+        w.il.C = c.take<double>((size_t)r * r);
+        w.il.Ci = c.take<double>((size_t)r * r);
     } else {
         std::memset(&w.il, 0, sizeof(w.il));
     }
@@ -171,6 +171,8 @@ GPTQ_API const char *gptq_status_string(int status) {
         default: return "unknown gptq status";
     }
 }
+
+GPTQ_API uint64_t gptq_launch_count(void) { return launch_counter().load(); }
 
 GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return GPTQ_ERR_CUDA;

@@ -16,6 +16,8 @@
 //   3. The sweep on [W, 0] with those n rows; R = the final extra columns, transposed.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "factor.cuh"
@@ -183,12 +185,12 @@ __global__ void sign_fix_kernel(float *V, int n, int r) {
 }
 
 // l~ = lambda_rel * (sum diag H + sum diag C) / (n + r); then C += l~ I.
-__global__ void il_lambda_kernel(const float *H, long long ldh, int n, float *C, int r,
+__global__ void il_lambda_kernel(const float *H, long long ldh, int n, double *C, int r,
                                  float lambda_rel, float *lam) {
     __shared__ double part[32];
     double acc = 0.0;
     for (int i = threadIdx.x; i < n + r; i += blockDim.x) {
-        const float d = i < n ? H[(long long)i * ldh + i] : C[(i - n) * r + (i - n)];
+        const double d = i < n ? (double)H[(long long)i * ldh + i] : C[(i - n) * r + (i - n)];
         if (i < n && !isfinite(d)) report(GPTQ_ERR_NONFINITE, (long long)i * ldh + i);
         acc += d;
     }
@@ -203,21 +205,22 @@ __global__ void il_lambda_kernel(const float *H, long long ldh, int n, float *C,
     __syncthreads();
     const float l = (float)((double)lambda_rel * part[0] / (double)(n + r));
     if (threadIdx.x == 0) *lam = l;
-    for (int i = threadIdx.x; i < r; i += blockDim.x) C[i * r + i] += l;
+    for (int i = threadIdx.x; i < r; i += blockDim.x) C[i * r + i] += (double)l;
 }
 
 struct ILWork {
-    float *Y, *Z, *G, *Gi, *Tm, *Qsel, *ev;   // subspace iteration
-    float *B12, *C, *Ci, *Y1, *Yr;            // Schur pieces
+    float *Y, *Z, *Tm, *Qsel, *ev;   // subspace iteration (n x p blocks, p x p Ritz matrix)
+    double *G, *Gi;                  // p x p Gram and inverse UL factor (fp64)
+    float *B12, *Y1, *Yr;            // n x r Schur pieces
+    double *C, *Ci;                  // r x r extra block and inverse UL factor (fp64)
 };
 
-inline int small_ul_inverse(float *M, float *Mi, int p, cudaStream_t s) {
-    // p <= FACTOR_NB: M = Ubar Ubar^T, Mi = Ubar^-1 (diag kernel; errors here are reported
-    // like any other non-positive pivot)
-    const int smem = 2 * FACTOR_NB * (FACTOR_NB + 1) * (int)sizeof(float);
-    cudaFuncSetAttribute(diag_ul_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    diag_ul_kernel<<<1, 512, smem, s>>>(M, p, Mi, p, 0, p);
-    return launch_status();
+// dst = src (src^T src)^-1/2-like, with the Gram, its factor and the product in fp64:
+// src^T src = Ubar Ubar^T, dst = src Ubar^-T has orthonormal columns.
+inline int cholqr_f64(const float *src, float *dst, int n, int p, ILWork &w, cudaStream_t s) {
+    if (int st = gemm_f64acc<float, float, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0, s)) return st;
+    if (int st = diag_ul_inv<double>(w.G, p, w.Gi, p, p, 0, s)) return st;
+    return gemm_f64acc<float, double, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.0, s);
 }
 
 // Top-r eigenvectors of H (n x n) into V (n x r).
@@ -227,19 +230,11 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
     random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
     GPTQ_CHECK_LAUNCH();
     for (int it = 0; it < IL_ITERS; ++it) {
-        // Z = H Y
+        // Z = H Y, then CholeskyQR2 (fp64 Gram): Y <- orth(Z)
         if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
-        // CholeskyQR2: Y = Z (Z^T Z)^-1/2-ish, twice
-        for (int pass = 0; pass < 2; ++pass) {
-            const float *src = pass == 0 ? w.Z : w.Y;
-            float *dst = pass == 0 ? w.Y : w.Z;
-            if (int st = gemm_simt(gemm_args<float, float>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.f, 0.f), s)) return st;
-            if (int st = small_ul_inverse(w.G, w.Gi, p, s)) return st;
-            // G = Ubar Ubar^T: src = (src Ubar^-T) Ubar^T, and src Ubar^-T has orthonormal columns
-            if (int st = gemm_simt(gemm_args<float, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.f, 0.f), s)) return st;
-        }
-        // the orthonormal block is now in Z; move it to Y
-        cudaMemcpyAsync(w.Y, w.Z, sizeof(float) * (size_t)n * p, cudaMemcpyDeviceToDevice, s);
+        if (int st = cholqr_f64(w.Z, w.Y, n, p, w, s)) return st;
+        if (int st = cholqr_f64(w.Y, w.Z, n, p, w, s)) return st;
+        std::swap(w.Y, w.Z);
     }
     // Rayleigh-Ritz: Tm = Y^T H Y
     if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
@@ -260,20 +255,16 @@ inline int il_factor(const float *H, long long ldh, int n, int r, const float *V
                      float lambda_rel, float *Uaug, float *Awork, float *T, float *lam,
                      ILWork &w, cudaStream_t s) {
     const long long ldu = n + r;
-    // B12 = H V (n x r), C = V^T B12 (r x r)
+    // B12 = H V (n x r), C = V^T B12 (r x r, fp64)
     if (int st = gemm_simt(gemm_args<float, float>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.f, 0.f), s)) return st;
-    if (int st = gemm_simt(gemm_args<float, float>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.f, 0.f), s)) return st;
+    if (int st = gemm_f64acc<float, float, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0, s)) return st;
     il_lambda_kernel<<<1, 1024, 0, s>>>(H, ldh, n, w.C, r, lambda_rel, lam);
     GPTQ_CHECK_LAUNCH();
-    // C = Ubar Ubar^T, Ci = Ubar^-1 ; C^-1 = Ci^T Ci
-    if (int st = small_ul_inverse(w.C, w.Ci, r, s)) return st;
+    // C = Ubar Ubar^T, Ci = Ubar^-1, C^-1 = Ci^T Ci
+    if (int st = diag_ul_inv<double>(w.C, r, w.Ci, r, r, 0, s)) return st;
     // Y1 = B12 Ci^T (n x r);  S = H + l I - Y1 Y1^T ; Yr = Y1 Ci = B12 C^-1
-    if (int st = gemm_simt(gemm_args<float, float>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.f, 0.f), s)) return st;
-    {
-        auto p = gemm_args<float, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.f, 0.f);
-        p.b_upper = 1;
-        if (int st = gemm_simt(p, s)) return st;
-    }
+    if (int st = gemm_f64acc<float, double, float>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, double, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.0, s, 1)) return st;
     copy_damped_kernel<<<1184, 256, 0, s>>>(H, ldh, Awork, n, n, lam);
     GPTQ_CHECK_LAUNCH();
     {

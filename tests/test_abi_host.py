@@ -18,7 +18,7 @@ def _declared():
 
 def test_header_declares_the_boundary():
     assert _declared() == sorted([
-        "gptq_workspace_size", "gptq_status_string", "gptq_sync_status",
+        "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
         "gptq_il_quantize_layer"])
 
@@ -85,7 +85,10 @@ def test_hessian_rejects_bad_arguments(args):
 
 
 def test_hessian_k0_is_a_noop():
+    import post_weight_quantization_06_b200 as g
+    before = g.gptq_launch_count()
     assert _lib().gptq_hessian_accumulate(P, P, 0, 0, 64, NULL) == 0
+    assert g.gptq_launch_count() == before
 
 
 @pytest.mark.parametrize("kw,expect", [

@@ -140,7 +140,7 @@ def test_quantize_stage_matches_oracle(g, m, n, bits, gs, B, wdt):
     uses the same fp32 values."""
     X = _spd_from_data(n, 4 * n, m + n + bits)
     Hd, _ = oracle.damp(oracle.hessian(X), 0.01)
-    U32 = oracle.inverse_cholesky_upper(Hd).astype(np.float32)
+    U32 = np.ascontiguousarray(oracle.inverse_cholesky_upper(Hd).astype(np.float32))
     W = torch.from_numpy(_rng(m * n).standard_normal((m, n)) * 0.02).float().to(DEV).to(wdt)
     G = n // gs if gs else 1
     codes = torch.empty(m, n * bits // 32, dtype=torch.int32, device=DEV)

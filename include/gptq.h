@@ -150,6 +150,35 @@ GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t 
                         size_t ws_bytes, gptq_stream_t stream);
 
 /*
+ * gptq_quantize_layer without a workspace argument and without any allocation.
+ * The pages have no counterpart to this entry point: it exists for callers that cannot
+ * hand the library device scratch memory, e.g. code running under a memory pool it does
+ * not own (a framework allocator that has reserved the device), or code that must not call
+ * cudaMalloc because it can synchronize the whole device and stall other work.
+ * It runs the same kernels as gptq_quantize_layer, with their scratch (the fp32 working
+ * copy of W and the per-panel errors) placed in a file-scope device array of
+ * GPTQ_NOALLOC_SCRATCH_BYTES bytes that every device loading the library holds until the
+ * process exits. The caller still provides W, U and the outputs, as for
+ * gptq_quantize_layer, and the arguments mean the same.
+ *   - Limit: gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size) must not exceed
+ *     GPTQ_NOALLOC_SCRATCH_BYTES (m * n + m * block_size floats, each part rounded up to
+ *     256 bytes; e.g. 2048 x 6144 fits); larger layers get GPTQ_ERR_ARG and nothing is
+ *     enqueued.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents behind. Calls
+ *     whose work overlaps on the GPU (other streams, other host threads) race on it:
+ *     serialise them. Nothing in the array needs to start at zero.
+ *   - Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+#define GPTQ_NOALLOC_SCRATCH_BYTES (64u << 20)
+GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
+                                         const float *U, int bits, int group_size,
+                                         int block_size, uint32_t *codes, float *scales,
+                                         uint8_t *zeros, double *loss_out,
+                                         gptq_stream_t stream);
+
+/*
  * GPTQ-intrinsic LoRA: quantize W against the augmented calibration X~ = [X, X V_r].
  * GPTQ-intrinsic LoRA summary, "Method" part 2: V_r (= L) are the top-r right singular
  * vectors of X; the pass runs on W~ = [W, 0] (r extra zero-initialised coordinates per

@@ -22,7 +22,7 @@ GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-            "gptq_il_quantize_layer")
+            "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer")
 
 
 class GptqError(RuntimeError):
@@ -46,6 +46,8 @@ def _load() -> ctypes.CDLL:
         "gptq_prepare_hinv": (c_int, [c_p, c_i64, c_f, c_p, c_p, c_p, c_sz, c_p]),
         "gptq_quantize_layer": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int,
                                         c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "gptq_quantize_layer_noalloc": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int,
+                                                c_int, c_p, c_p, c_p, c_p, c_p]),
         "gptq_il_quantize_layer": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int,
                                            c_f, c_int, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
                                            c_sz, c_p]),
@@ -154,6 +156,29 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, bits: int, group_size:
                                     block_size, _ptr(codes), _ptr(scales), _ptr(zeros),
                                     _ptr(loss_out), _ptr(ws), ws.numel(), _stream(stream)),
            "gptq_quantize_layer")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def gptq_quantize_layer_noalloc(W: torch.Tensor, U: torch.Tensor, bits: int, group_size: int,
+                                block_size: int, codes: torch.Tensor, scales: torch.Tensor,
+                                zeros: torch.Tensor, loss_out: torch.Tensor | None, stream=None):
+    """gptq_quantize_layer for callers that cannot provide device scratch memory: the
+    library's own fixed device array (NOALLOC_SCRATCH_BYTES) is used instead, shared by every
+    call on the device, so overlapping calls must be serialised by the caller."""
+    _dev(W, "W")
+    _dev(U, "U", torch.float32)
+    _dev(codes, "codes", torch.int32)
+    _dev(scales, "scales", torch.float32)
+    _dev(zeros, "zeros", torch.uint8)
+    if loss_out is not None:
+        _dev(loss_out, "loss_out", torch.float64)
+    m, n = W.shape
+    _check(_lib.gptq_quantize_layer_noalloc(_ptr(W), _dtype_code(W), m, n, _ptr(U), bits,
+                                            group_size, block_size, _ptr(codes), _ptr(scales),
+                                            _ptr(zeros), _ptr(loss_out), _stream(stream)),
+           "gptq_quantize_layer_noalloc")
 
 
 def gptq_il_quantize_layer(W: torch.Tensor, H: torch.Tensor, r: int, bits: int, group_size: int,

@@ -1,6 +1,7 @@
 // libgptq: C ABI of the GPTQ / GPTQ-intrinsic-LoRA layer pass for sm_100a.
 // One translation unit: the kernels live in the included .cuh files.
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
@@ -131,6 +132,32 @@ int init_work(const void *W, int w_dtype, long long m, int n, float *Wc, long lo
     return launch_status();
 }
 
+// ---------------------------------------------------------------------------------------
+// Scratch for gptq_quantize_layer_noalloc: a fixed file-scope device array, so that the
+// entry point needs neither a workspace from the caller nor any allocation. Every device
+// that loads the library holds it until the process exits. In host code the symbol is only a
+// stand-in; its device address is looked up once per device (noalloc_scratch()).
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GPTQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+static void *g_noalloc_ptr[kMaxDevices];
+static std::mutex g_noalloc_mutex;
+
+// Device address of g_noalloc_scratch on the current device (looked up on the first call per
+// device), or nullptr if the lookup fails.
+inline void *noalloc_scratch() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_ptr[dev] = p;
+    }
+    return g_noalloc_ptr[dev];
+}
+
 }  // namespace gptq
 
 using namespace gptq;
@@ -219,6 +246,28 @@ GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t 
     if (int st = check_ws(workspace, ws_bytes, need)) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     Carver c(workspace);
+    QuantWs w = carve_quant(c, m, n, block_size);
+    if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
+    return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
+                       codes, scales, zeros, loss_out, w.Err, s);
+}
+
+GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
+                                         const float *U, int bits, int group_size,
+                                         int block_size, uint32_t *codes, float *scales,
+                                         uint8_t *zeros, double *loss_out,
+                                         gptq_stream_t stream) {
+    if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (!valid_quant_args(m, n, bits, group_size, block_size)) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size);
+    if (need > GPTQ_NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
+    void *scratch = noalloc_scratch();
+    if (!scratch) return GPTQ_ERR_CUDA;
+    // The working copy and the per-panel errors are fully written before they are read, so
+    // nothing left in the shared scratch by an earlier call needs clearing.
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(scratch);
     QuantWs w = carve_quant(c, m, n, block_size);
     if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
     return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,

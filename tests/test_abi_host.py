@@ -20,7 +20,7 @@ def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-        "gptq_il_quantize_layer"])
+        "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer"])
 
 
 def test_library_exports_every_declared_symbol():

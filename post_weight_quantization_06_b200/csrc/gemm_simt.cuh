@@ -128,19 +128,32 @@ template <> __device__ __forceinline__ double to_f64<__nv_bfloat16>(__nv_bfloat1
     return (double)__bfloat162float(x);
 }
 
-// C = alpha * op(A) op(B) accumulated in fp64 (64 x 64 tiles, 4 x 4 per thread). For the
-// small and skinny products of the orthonormalisation steps, where fp32 accumulation would
-// lose the weak directions of an ill-conditioned block.
+// Optional epilogue of the fp64-accumulating GEMM:
+//   C(i,j) = alpha * acc + beta * Cin(i,j) + (i == j ? *diag : 0), written only for j >= i
+//   when c_upper is set. Cin may alias C.
+struct F64Epilogue {
+    const float *Cin = nullptr;
+    long long ldcin = 0;
+    double beta = 0.0;
+    const float *diag = nullptr;
+    int c_upper = 0;
+};
+
+// C = alpha * op(A) op(B) (+ epilogue) accumulated in fp64 (64 x 64 tiles, 4 x 4 per thread).
+// For the products whose result is a small difference of large numbers or must keep the weak
+// directions of an ill-conditioned block: the orthonormalisation and Rayleigh-Ritz steps and
+// the Schur complement of the intrinsic-LoRA factor.
 template <typename TA, typename TB, typename TC>
 __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, const TA *A,
                                                           long long lda, int ta, const TB *B,
                                                           long long ldb, int tb, TC *C,
                                                           long long ldc, double alpha,
-                                                          int b_upper) {
+                                                          int b_upper, F64Epilogue ep) {
     constexpr int T = 64, BK = 16;
     __shared__ double As[BK][T + 1];
     __shared__ double Bs[BK][T + 1];
     const int i0 = blockIdx.y * T, j0 = blockIdx.x * T;
+    if (ep.c_upper && i0 >= j0 + T) return;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     double acc[4][4] = {};
     int kend = K;
@@ -174,6 +187,7 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
         }
         __syncthreads();
     }
+    const double dg = ep.diag ? (double)*ep.diag : 0.0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         const int gi = i0 + ty + 16 * u;
@@ -181,7 +195,11 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const int gj = j0 + tx + 16 * v;
-            if (gj < N) C[(long long)gi * ldc + gj] = (TC)(alpha * acc[u][v]);
+            if (gj >= N || (ep.c_upper && gj < gi)) continue;
+            double val = alpha * acc[u][v];
+            if (ep.Cin) val += ep.beta * (double)ep.Cin[(long long)gi * ep.ldcin + gj];
+            if (gi == gj) val += dg;
+            C[(long long)gi * ldc + gj] = (TC)val;
         }
     }
 }
@@ -189,11 +207,11 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
 template <typename TA, typename TB, typename TC>
 inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, const TB *B,
                        long long ldb, int tb, TC *C, long long ldc, double alpha, cudaStream_t s,
-                       int b_upper = 0) {
+                       int b_upper = 0, F64Epilogue ep = F64Epilogue()) {
     if (M <= 0 || N <= 0) return GPTQ_OK;
     dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
     gemm_f64acc_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, lda, ta, B, ldb, tb, C, ldc,
-                                                        alpha, b_upper);
+                                                        alpha, b_upper, ep);
     return launch_status();
 }
 

@@ -8,6 +8,7 @@
 #include "factor.cuh"
 #include "quant.cuh"
 #include "il.cuh"
+#include "hessian_tc.cuh"
 
 namespace gptq {
 
@@ -63,13 +64,14 @@ inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
         const int p = il_block_p((int)n, r);
         w.il.Y = c.take<float>((size_t)n * p);
         w.il.Z = c.take<float>((size_t)n * p);
-        w.il.Tm = c.take<float>((size_t)p * p);
         w.il.Qsel = c.take<float>((size_t)p * r);
-        w.il.ev = c.take<float>((size_t)p);
+        w.il.HY = c.take<double>((size_t)n * p);
+        w.il.Tm = c.take<double>((size_t)p * p);
+        w.il.ev = c.take<double>((size_t)p);
         w.il.G = c.take<double>((size_t)p * p);
         w.il.Gi = c.take<double>((size_t)p * p);
-        w.il.B12 = c.take<float>((size_t)n * r);
-        w.il.Y1 = c.take<float>((size_t)n * r);
+        w.il.B12 = c.take<double>((size_t)n * r);
+        w.il.Y1 = c.take<double>((size_t)n * r);
         w.il.Yr = c.take<float>((size_t)n * r);
         w.il.C = c.take<double>((size_t)r * r);
         w.il.Ci = c.take<double>((size_t)r * r);
@@ -217,8 +219,14 @@ GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64
     if (x_dtype != GPTQ_BF16 && x_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
     if (k == 0) return GPTQ_OK;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (x_dtype == GPTQ_BF16)
-        return hessian_simt(H, static_cast<const __nv_bfloat16 *>(X), k, (int)n, s);
+    if (x_dtype == GPTQ_BF16) {
+        const auto *Xb = static_cast<const __nv_bfloat16 *>(X);
+        // tensor-core path: TMA needs a 16-byte aligned base and 16-byte row pitch
+        if (n % 8 == 0 && (reinterpret_cast<uintptr_t>(X) & 15u) == 0 &&
+            std::getenv("GPTQ_FORCE_SIMT_HESSIAN") == nullptr)
+            return tc::hessian_tc(H, Xb, k, (int)n, s);
+        return hessian_simt(H, Xb, k, (int)n, s);
+    }
     return hessian_simt(H, static_cast<const float *>(X), k, (int)n, s);
 }
 

@@ -25,7 +25,6 @@
 namespace gptq {
 
 constexpr int IL_MAX_R = 128;
-constexpr int IL_ITERS = 6;
 
 inline int il_block_p(int n, int r) {
     int p = r + 32 > 2 * r ? r + 32 : 2 * r;
@@ -53,99 +52,90 @@ __global__ void random_block_kernel(float *Y, long long total, unsigned long lon
 }
 
 // One-CTA cyclic Jacobi on a symmetric p x p matrix (p even, p <= 128), round-robin
-// ordering so that p/2 disjoint rotations run at once. On exit: eigenvalues on the
-// diagonal of T; eigenvectors in the columns of Q. Then the r largest are selected in
-// decreasing order: evals[0..r), Qsel (p x r, column c = eigenvector of the c-th largest).
-__global__ __launch_bounds__(512) void jacobi_eig_kernel(const float *Tin, int p, int r,
-                                                         float *Qsel, float *evals) {
-    extern __shared__ float sm[];
+// ordering so that p/2 disjoint rotations run at once. The matrix is held in fp64, the
+// accumulated rotations in fp32 (both in shared memory). On exit the r largest eigenvalues
+// are written in decreasing order to evals[0..r) and their eigenvectors to the columns of
+// Qsel (p x r).
+__global__ __launch_bounds__(512) void jacobi_eig_kernel(const double *Tin, int p, int r,
+                                                         float *Qsel, double *evals) {
+    extern __shared__ __align__(16) unsigned char jsm[];
     const int LD = p + 1;
-    float *T = sm;
-    float *Q = T + p * LD;
-    float *cs = Q + p * LD;       // p/2 cosines
-    float *sn = cs + p / 2;       // p/2 sines
-    int *pi = reinterpret_cast<int *>(sn + p / 2);
+    double *T = reinterpret_cast<double *>(jsm);
+    double *cs = T + p * LD;      // p/2 cosines
+    double *sn = cs + p / 2;      // p/2 sines
+    float *Q = reinterpret_cast<float *>(sn + p / 2);
+    int *pi = reinterpret_cast<int *>(Q + p * LD);
     int *pj = pi + p / 2;
-    __shared__ float off_s;
+    __shared__ double red[2];
     const int tid = threadIdx.x, nt = blockDim.x;
     for (int idx = tid; idx < p * p; idx += nt) {
         const int i = idx / p, j = idx % p;
-        T[i * LD + j] = 0.5f * (Tin[i * p + j] + Tin[j * p + i]);
+        T[i * LD + j] = 0.5 * (Tin[i * p + j] + Tin[j * p + i]);
         Q[i * LD + j] = (i == j) ? 1.f : 0.f;
     }
-    __syncthreads();
     const int half = p / 2;
-    for (int sweep = 0; sweep < 15; ++sweep) {
-        // off-diagonal mass relative to the diagonal
-        if (tid == 0) off_s = 0.f;
+    for (int sweep = 0; sweep < 20; ++sweep) {
+        if (tid < 2) red[tid] = 0.0;
         __syncthreads();
-        float loc = 0.f, dg = 0.f;
+        double off = 0.0, dia = 0.0;
         for (int idx = tid; idx < p * p; idx += nt) {
             const int i = idx / p, j = idx % p;
-            const float v = T[i * LD + j];
-            if (i != j) loc += v * v; else dg += v * v;
+            const double v = T[i * LD + j];
+            if (i != j) off += v * v; else dia += v * v;
         }
-        atomicAdd(&off_s, loc);
+        off = warp_sum_d(off);
+        dia = warp_sum_d(dia);
+        if ((tid & 31) == 0) { atomicAdd(&red[0], off); atomicAdd(&red[1], dia); }
         __syncthreads();
-        const float off = off_s;
+        const bool done = red[0] <= 1e-26 * red[1];
         __syncthreads();
-        if (tid == 0) off_s = 0.f;
-        __syncthreads();
-        atomicAdd(&off_s, dg);
-        __syncthreads();
-        const float dia = off_s;
-        __syncthreads();
-        if (off <= 1e-10f * dia) break;
+        if (done) break;
         for (int rnd = 0; rnd < p - 1; ++rnd) {
             for (int k = tid; k < half; k += nt) {
-                // circle method: position 0 fixed, positions 1..p-1 rotate
-                const int xa = k, xb = p - 1 - k;
-                const int a = xa == 0 ? 0 : 1 + (xa - 1 + rnd) % (p - 1);
+                const int xb = p - 1 - k;
+                const int a = k == 0 ? 0 : 1 + (k - 1 + rnd) % (p - 1);
                 const int b = 1 + (xb - 1 + rnd) % (p - 1);
                 const int i = min(a, b), j = max(a, b);
                 pi[k] = i; pj[k] = j;
-                const float aij = T[i * LD + j];
-                float c = 1.f, s = 0.f;
-                if (aij != 0.f) {
-                    const float tau = (T[j * LD + j] - T[i * LD + i]) / (2.f * aij);
-                    const float t = (tau >= 0.f ? 1.f : -1.f) / (fabsf(tau) + sqrtf(1.f + tau * tau));
-                    c = rsqrtf(1.f + t * t);
-                    s = t * c;
+                const double aij = T[i * LD + j];
+                double c = 1.0, sv = 0.0;
+                if (aij != 0.0) {
+                    const double tau = (T[j * LD + j] - T[i * LD + i]) / (2.0 * aij);
+                    const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
+                    c = 1.0 / sqrt(1.0 + t * t);
+                    sv = t * c;
                 }
-                cs[k] = c; sn[k] = s;
+                cs[k] = c; sn[k] = sv;
             }
             __syncthreads();
-            // rows: row_i <- c row_i - s row_j ; row_j <- s row_i + c row_j
             for (int idx = tid; idx < half * p; idx += nt) {
                 const int k = idx / p, l = idx % p;
                 const int i = pi[k], j = pj[k];
-                const float c = cs[k], s = sn[k];
-                const float ti = T[i * LD + l], tj = T[j * LD + l];
-                T[i * LD + l] = c * ti - s * tj;
-                T[j * LD + l] = s * ti + c * tj;
+                const double c = cs[k], sv = sn[k];
+                const double ti = T[i * LD + l], tj = T[j * LD + l];
+                T[i * LD + l] = c * ti - sv * tj;
+                T[j * LD + l] = sv * ti + c * tj;
             }
             __syncthreads();
-            // columns of T and of Q
             for (int idx = tid; idx < half * p; idx += nt) {
                 const int k = idx / p, l = idx % p;
                 const int i = pi[k], j = pj[k];
-                const float c = cs[k], s = sn[k];
-                const float ti = T[l * LD + i], tj = T[l * LD + j];
-                T[l * LD + i] = c * ti - s * tj;
-                T[l * LD + j] = s * ti + c * tj;
+                const double c = cs[k], sv = sn[k];
+                const double ti = T[l * LD + i], tj = T[l * LD + j];
+                T[l * LD + i] = c * ti - sv * tj;
+                T[l * LD + j] = sv * ti + c * tj;
                 const float qi = Q[l * LD + i], qj = Q[l * LD + j];
-                Q[l * LD + i] = c * qi - s * qj;
-                Q[l * LD + j] = s * qi + c * qj;
+                Q[l * LD + i] = (float)(c * qi - sv * qj);
+                Q[l * LD + j] = (float)(sv * qi + c * qj);
             }
             __syncthreads();
         }
     }
-    // rank by decreasing eigenvalue (ties by index)
     for (int i = tid; i < p; i += nt) {
-        const float li = T[i * LD + i];
+        const double li = T[i * LD + i];
         int rank = 0;
         for (int j = 0; j < p; ++j) {
-            const float lj = T[j * LD + j];
+            const double lj = T[j * LD + j];
             rank += (lj > li) || (lj == li && j < i);
         }
         if (rank < r) {
@@ -153,6 +143,11 @@ __global__ __launch_bounds__(512) void jacobi_eig_kernel(const float *Tin, int p
             for (int l = 0; l < p; ++l) Qsel[l * r + rank] = Q[l * LD + i];
         }
     }
+}
+
+inline size_t jacobi_smem(int p) {
+    return (size_t)p * (p + 1) * sizeof(double) + (size_t)p * sizeof(double) +
+           (size_t)p * (p + 1) * sizeof(float) + (size_t)p * sizeof(int);
 }
 
 // Columns of V (n x r): flip so that the largest-magnitude entry (first on ties) is positive.
@@ -209,14 +204,19 @@ __global__ void il_lambda_kernel(const float *H, long long ldh, int n, double *C
 }
 
 struct ILWork {
-    float *Y, *Z, *Tm, *Qsel, *ev;   // subspace iteration (n x p blocks, p x p Ritz matrix)
-    double *G, *Gi;                  // p x p Gram and inverse UL factor (fp64)
-    float *B12, *Y1, *Yr;            // n x r Schur pieces
-    double *C, *Ci;                  // r x r extra block and inverse UL factor (fp64)
+    float *Y, *Z, *Qsel;       // subspace iteration blocks (n x p) and selected Ritz vectors
+    double *HY, *Tm, *ev;      // fp64 Rayleigh-Ritz: H Y (n x p), Y^T H Y (p x p), values
+    double *G, *Gi;            // p x p Gram and inverse UL factor
+    double *B12, *Y1;          // n x r: H V and H V C^-1/2
+    float *Yr;                 // n x r: H V C^-1
+    double *C, *Ci;            // r x r extra block and inverse UL factor
 };
 
-// dst = src (src^T src)^-1/2-like, with the Gram, its factor and the product in fp64:
-// src^T src = Ubar Ubar^T, dst = src Ubar^-T has orthonormal columns.
+constexpr int IL_ITERS_F32 = 4;   // power steps with fp32 accumulation
+constexpr int IL_ITERS_F64 = 1;   // then with fp64 accumulation, before Rayleigh-Ritz
+
+// dst = src Ubar^-T where src^T src = Ubar Ubar^T (Gram, factor and product in fp64):
+// dst has orthonormal columns spanning src.
 inline int cholqr_f64(const float *src, float *dst, int n, int p, ILWork &w, cudaStream_t s) {
     if (int st = gemm_f64acc<float, float, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0, s)) return st;
     if (int st = diag_ul_inv<double>(w.G, p, w.Gi, p, p, 0, s)) return st;
@@ -229,49 +229,53 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
     const int p = il_block_p(n, r);
     random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
     GPTQ_CHECK_LAUNCH();
-    for (int it = 0; it < IL_ITERS; ++it) {
-        // Z = H Y, then CholeskyQR2 (fp64 Gram): Y <- orth(Z)
-        if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
+    for (int it = 0; it < IL_ITERS_F32 + IL_ITERS_F64; ++it) {
+        // Z = H Y, then CholeskyQR2: Y <- orth(Z)
+        if (it < IL_ITERS_F32) {
+            if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
+        } else {
+            if (int st = gemm_f64acc<float, float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.0, s)) return st;
+        }
         if (int st = cholqr_f64(w.Z, w.Y, n, p, w, s)) return st;
         if (int st = cholqr_f64(w.Y, w.Z, n, p, w, s)) return st;
         std::swap(w.Y, w.Z);
     }
-    // Rayleigh-Ritz: Tm = Y^T H Y
-    if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
-    if (int st = gemm_simt(gemm_args<float, float>(p, p, n, w.Y, p, 1, w.Z, p, 0, w.Tm, p, 1.f, 0.f), s)) return st;
-    const int smem = (2 * p * (p + 1) + 2 * p) * (int)sizeof(float);
-    cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // Rayleigh-Ritz in fp64: Tm = Y^T (H Y)
+    if (int st = gemm_f64acc<float, float, double>(n, p, n, H, ldh, 0, w.Y, p, 0, w.HY, p, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p, 1.0, s)) return st;
+    const size_t smem = jacobi_smem(p);
+    cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     jacobi_eig_kernel<<<1, 512, smem, s>>>(w.Tm, p, r, w.Qsel, w.ev);
     GPTQ_CHECK_LAUNCH();
     // V = Y Qsel
-    if (int st = gemm_simt(gemm_args<float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.f, 0.f), s)) return st;
+    if (int st = gemm_f64acc<float, float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.0, s)) return st;
     sign_fix_kernel<<<r, 256, 0, s>>>(V, n, r);
     return launch_status();
 }
 
 // First n rows of U~ into Uaug (n x (n + r), ldu = n + r), lambda~ into *lam.
+// The Schur complement S = H + l I - H V C^-1 V^T H cancels the large eigenvalues of H along
+// V down to about l; it is formed with fp64 accumulation from the fp32 H and V, and only the
+// (well conditioned) result is rounded to fp32 for the factor.
 // Awork: n x n scratch, T: FACTOR_NB x n scratch.
 inline int il_factor(const float *H, long long ldh, int n, int r, const float *V,
                      float lambda_rel, float *Uaug, float *Awork, float *T, float *lam,
                      ILWork &w, cudaStream_t s) {
     const long long ldu = n + r;
-    // B12 = H V (n x r), C = V^T B12 (r x r, fp64)
-    if (int st = gemm_simt(gemm_args<float, float>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.f, 0.f), s)) return st;
-    if (int st = gemm_f64acc<float, float, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0, s)) return st;
+    // B12 = H V (n x r), C = V^T B12 (r x r)
+    if (int st = gemm_f64acc<float, float, double>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, double, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0, s)) return st;
     il_lambda_kernel<<<1, 1024, 0, s>>>(H, ldh, n, w.C, r, lambda_rel, lam);
     GPTQ_CHECK_LAUNCH();
     // C = Ubar Ubar^T, Ci = Ubar^-1, C^-1 = Ci^T Ci
     if (int st = diag_ul_inv<double>(w.C, r, w.Ci, r, r, 0, s)) return st;
-    // Y1 = B12 Ci^T (n x r);  S = H + l I - Y1 Y1^T ; Yr = Y1 Ci = B12 C^-1
-    if (int st = gemm_f64acc<float, double, float>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.0, s)) return st;
-    if (int st = gemm_f64acc<float, double, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.0, s, 1)) return st;
-    copy_damped_kernel<<<1184, 256, 0, s>>>(H, ldh, Awork, n, n, lam);
-    GPTQ_CHECK_LAUNCH();
-    {
-        auto p = gemm_args<float, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.f, 1.f);
-        p.c_upper = 1;
-        if (int st = gemm_simt(p, s)) return st;
-    }
+    // Y1 = B12 Ci^T, Yr = Y1 Ci = B12 C^-1
+    if (int st = gemm_f64acc<double, double, double>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.0, s)) return st;
+    if (int st = gemm_f64acc<double, double, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.0, s, 1)) return st;
+    // S = H + l I - Y1 Y1^T (upper triangle), fp64 accumulation, fp32 result
+    F64Epilogue ep;
+    ep.Cin = H; ep.ldcin = ldh; ep.beta = 1.0; ep.diag = lam; ep.c_upper = 1;
+    if (int st = gemm_f64acc<double, double, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.0, s, 0, ep)) return st;
     cudaMemsetAsync(Uaug, 0, sizeof(float) * (size_t)n * ldu, s);
     if (int st = factor_ul_inverse(Awork, n, Uaug, ldu, n, T, s)) return st;
     // U12 = -U11 Yr

@@ -64,6 +64,44 @@ def test_hessian_bf16(g, n, k, chunks):
     assert torch.equal(H, H.t())
 
 
+@pytest.mark.parametrize("n,k", [(512, 20000), (1536, 65536)])
+def test_hessian_tensor_core_path_is_tighter_than_fp32_chain(g, n, k, monkeypatch):
+    """bf16 X with n % 8 == 0 runs on tcgen05 with compensated chunk sums; the SIMT path
+    (forced by GPTQ_FORCE_SIMT_HESSIAN) is a plain fp32 chain. Both against the oracle."""
+    X = torch.from_numpy(_spd_from_data(n, k, 3 * n)).float().to(DEV).to(torch.bfloat16)
+    Href = oracle.hessian(np64(X))
+    H_tc = torch.zeros(n, n, device=DEV)
+    g.gptq_hessian_accumulate(H_tc, X)
+    g.gptq_sync_status()
+    monkeypatch.setenv("GPTQ_FORCE_SIMT_HESSIAN", "1")
+    H_simt = torch.zeros(n, n, device=DEV)
+    g.gptq_hessian_accumulate(H_simt, X)
+    g.gptq_sync_status()
+    e_tc, e_simt = rel_fro(np64(H_tc), Href), rel_fro(np64(H_simt), Href)
+    print(f"H n={n} k={k}: tensor-core rel err {e_tc:.2e}, SIMT rel err {e_simt:.2e}")
+    assert torch.equal(H_tc, H_tc.t())
+    assert e_tc <= REL_H and e_tc <= e_simt
+
+
+def test_hessian_bounded_wait_reports_timeout_and_device_stays_usable(g, monkeypatch):
+    """A wait that nothing will ever satisfy (test hook) gives up after the limit, reports
+    GPTQ_ERR_TIMEOUT through the status word, and the next call works normally."""
+    n, k = 256, 4096
+    X = torch.from_numpy(_spd_from_data(n, k, 11)).float().to(DEV).to(torch.bfloat16)
+    monkeypatch.setenv("GPTQ_TEST_STALL", "1")
+    monkeypatch.setenv("GPTQ_WAIT_LIMIT_CYCLES", "2000000")
+    H = torch.zeros(n, n, device=DEV)
+    g.gptq_hessian_accumulate(H, X)
+    st, info = g.gptq_sync_status(raise_on_error=False)
+    assert st == g.GPTQ_ERR_TIMEOUT and info in (1, 2, 3, 4, 5)
+    monkeypatch.delenv("GPTQ_TEST_STALL")
+    monkeypatch.delenv("GPTQ_WAIT_LIMIT_CYCLES")
+    H.zero_()
+    g.gptq_hessian_accumulate(H, X)
+    g.gptq_sync_status()
+    assert rel_fro(np64(H), oracle.hessian(np64(X))) <= REL_H
+
+
 # ----------------------------------------------------------------------------- factor
 
 @pytest.mark.parametrize("n,k,lam", [(256, 512, 0.01), (300, 2000, 0.01), (1024, 4096, 0.01),

@@ -48,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="use only the first TOKENS calibration rows (small profiling cases)")
     return ap.parse_args(argv)
 
 
@@ -320,6 +322,9 @@ def bench_ours(args):
     import post_weight_quantization_06_b200 as g
 
     layer = datagen.WORKLOADS[args.workload](device=dev, seed=rank_seed(args.workload, rank))
+    if args.tokens:
+        layer.X = layer.X[: args.tokens].clone()
+        torch.cuda.empty_cache()
     stream = torch.cuda.Stream(device=dev)
     lp = LayerPass(g, layer, stream)
     for _ in range(args.warmup):

@@ -8,87 +8,125 @@
 // Then U^T U = Ubar^-T Ubar^-1 = A^-1, and since the upper factor of A^-1 with a positive
 // diagonal is unique, this is the U of the chol -> inverse -> chol route.
 //
-// Blocked, bottom-right first, with blocks of NB columns. For block p (rows r0..r1):
-//   1. diag:  A_pp = Ubar_pp Ubar_pp^T  and  U_pp = Ubar_pp^-1          (one CTA)
-//      (Ubar_pp itself is used by no later step)
-//   2. panel: Ubar[0:r0, p] = A[0:r0, p] U_pp^T                           (GEMM)
-//   3. syrk:  A[0:r0, 0:r0] -= Ubar[0:r0, p] Ubar[0:r0, p]^T (upper)       (GEMM)
-//   4. row p of U:  U[p, r1:] = -U_pp (Ubar[p, r1:] U[r1:, r1:])          (two GEMMs)
-// Step 4 uses Ubar's row block p (finished by earlier, later-indexed blocks) and the
-// already finished trailing part of U.
+// Recursive, bottom-right half first (factor_rec below): the work is four large GEMMs per
+// split (tensor cores through gemm_f32) and one-CTA register-tiled kernels on the
+// 128-column diagonal leaves (diag_ul_inv_kernel).
 #pragma once
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 
 namespace gptq {
 
 constexpr int FACTOR_NB = 128;
 
-// One CTA: UL-Cholesky of an nb x nb symmetric block (upper triangle read) followed by the
-// inverse of its factor, in place in shared memory. On exit U's block holds
-// U_pp = Ubar_pp^-1 (upper; strictly lower part zeroed), where A_pp = Ubar_pp Ubar_pp^T.
-// Ubar_pp itself is not needed by any later step and is not stored.
-// Column c is processed from the last to the first: pivot, scaled column above it, update
-// of the leading block; then row c of the inverse, which only needs Ubar's row c (saved
-// first) and the rows of the inverse below it (already in place).
+// One CTA: UL-Cholesky of an nb x nb symmetric block (upper triangle read) and the inverse of
+// its factor. On exit U's block holds U_pp = Ubar_pp^-1 (upper; strictly lower part zeroed),
+// where A_pp = Ubar_pp Ubar_pp^T; Ubar_pp itself is used by no later step and is not stored.
+//
+// Register-tiled sweep: thread (ty, tx) of a 16 x 16 grid holds the 8 x 8 entries with rows
+// ty + 16 a and columns tx + 16 b of one matrix M. Before step c, M's columns <= c hold the
+// leading block still to be factored and its columns > c hold, for rows < c, the partial sums
+// P[i][j] = sum_{k > c} Ubar[i][k] X[k][j] of the inverse X = Ubar^-1 (rows > c of M already
+// are rows of X). Step c (from the last column to the first), with one barrier:
+//   column c (rows <= c) and row c (columns > c) of M are published to shared memory;
+//   pivot d = M[c][c], u_i = M[i][c] / sqrt(d) (Ubar's column c), row c of X is
+//   x_c = 1/sqrt(d), x_j = -P[c][j] / sqrt(d);
+//   rows i < c get M[i][j] += u_i v_j with v_j = -u_j (j < c: the Cholesky update),
+//   v_c = x_c (column c restarts as a partial sum), v_j = x_j (j > c: the inverse update).
 // A pivot <= 0 (or NaN) records GPTQ_ERR_NOT_PD with info = col_base + c and continues with a
 // unit pivot so that the kernel always finishes.
-template <typename T>
-__global__ __launch_bounds__(512) void diag_ul_inv_kernel(const T *A, long long lda, T *U,
-                                                          long long ldu, int nb,
-                                                          long long col_base) {
-    extern __shared__ __align__(16) unsigned char smraw[];
-    T *S = reinterpret_cast<T *>(smraw);
-    T *rowc = S + nb * (nb + 1);
-    const int LD = nb + 1;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
-        const int i = idx / nb, j = idx % nb;
-        S[i * LD + j] = (j >= i) ? A[(long long)i * lda + j] : T(0);
-    }
-    __syncthreads();
-    for (int c = nb - 1; c >= 0; --c) {
-        const T d = S[c * LD + c];
-        const bool bad = !(d > T(0)) || !isfinite((double)d);
-        if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
-        const T piv = bad ? T(1) : sqrt(d);
-        __syncthreads();
-        for (int i = tid; i < c; i += blockDim.x) S[i * LD + c] = S[i * LD + c] / piv;
-        for (int k = c + 1 + tid; k < nb; k += blockDim.x) rowc[k] = S[c * LD + k];
-        __syncthreads();
-        for (int i = warp; i < c; i += nw) {
-            const T sic = S[i * LD + c];
-            for (int j = i + lane; j < c; j += 32) S[i * LD + j] -= sic * S[j * LD + c];
-        }
-        const T xcc = T(1) / piv;
-        for (int j = c + 1 + warp; j < nb; j += nw) {
-            T acc = T(0);
-            for (int k = c + 1 + lane; k <= j; k += 32) acc += rowc[k] * S[k * LD + j];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-            if (lane == 0) S[c * LD + j] = -xcc * acc;
-        }
-        if (tid == 0) S[c * LD + c] = xcc;
-        __syncthreads();
-    }
-    for (int idx = tid; idx < nb * nb; idx += blockDim.x) {
-        const int i = idx / nb, j = idx % nb;
-        U[(long long)i * ldu + j] = (j >= i) ? S[i * LD + j] : T(0);
-    }
-}
+constexpr int DIAG_THREADS = 256;
 
 template <typename T>
-inline size_t diag_smem(int nb) { return ((size_t)nb * (nb + 1) + nb) * sizeof(T); }
+__global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, long long lda,
+                                                                   T *U, long long ldu, int nb,
+                                                                   long long col_base) {
+    __shared__ T colb[2][FACTOR_NB];
+    __shared__ T rowb[2][FACTOR_NB];
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    T M[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int i = ty + 16 * a, j = tx + 16 * b;
+            T v = T(0);
+            if (i < nb && j < nb) v = j >= i ? A[(long long)i * lda + j] : A[(long long)j * lda + i];
+            M[a][b] = v;
+        }
+    int buf = 0;
+#pragma unroll
+    for (int b = 7; b >= 0; --b) {
+        for (int cc = 15; cc >= 0; --cc) {
+            const int c = 16 * b + cc;
+            if (c >= nb) continue;
+            if (tx == cc) {
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    if (ty + 16 * a <= c) colb[buf][ty + 16 * a] = M[a][b];
+            }
+            if (ty == cc) {
+#pragma unroll
+                for (int b2 = 0; b2 < 8; ++b2) {
+                    const int j = tx + 16 * b2;
+                    if (j > c && j < nb) rowb[buf][j] = M[b][b2];
+                }
+            }
+            __syncthreads();
+            const T d = colb[buf][c];
+            const bool bad = !(d > T(0)) || !isfinite((double)d);
+            if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
+            const T ipiv = T(1) / (bad ? T(1) : sqrt(d));
+            T u[8], v[8];
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                const int i = ty + 16 * a;
+                u[a] = i < c ? colb[buf][i] * ipiv : T(0);
+            }
+#pragma unroll
+            for (int b2 = 0; b2 < 8; ++b2) {
+                const int j = tx + 16 * b2;
+                v[b2] = j < c ? -colb[buf][j] * ipiv
+                              : (j == c ? ipiv : (j < nb ? -ipiv * rowb[buf][j] : T(0)));
+            }
+            if (tx == cc) {
+#pragma unroll
+                for (int a = 0; a < 8; ++a)
+                    if (ty + 16 * a < c) M[a][b] = T(0);
+            }
+#pragma unroll
+            for (int a = 0; a < 8; ++a) {
+                if (ty + 16 * a < c) {
+#pragma unroll
+                    for (int b2 = 0; b2 < 8; ++b2) M[a][b2] = fma(u[a], v[b2], M[a][b2]);
+                }
+            }
+            if (ty == cc) {
+#pragma unroll
+                for (int b2 = 0; b2 < 8; ++b2) {
+                    const int j = tx + 16 * b2;
+                    if (j >= c && j < nb) M[b][b2] = v[b2];
+                }
+            }
+            buf ^= 1;
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int i = ty + 16 * a, j = tx + 16 * b;
+            if (i < nb && j < nb) U[(long long)i * ldu + j] = j >= i ? M[a][b] : T(0);
+        }
+}
 
 // U_pp = inverse of the UL factor of the nb x nb block at A (nb <= FACTOR_NB).
 template <typename T>
 inline int diag_ul_inv(const T *A, long long lda, T *U, long long ldu, int nb, long long col_base,
                        cudaStream_t s) {
-    const size_t smem = diag_smem<T>(FACTOR_NB);
-    cudaFuncSetAttribute(diag_ul_inv_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    diag_ul_inv_kernel<T><<<1, 512, diag_smem<T>(nb), s>>>(A, lda, U, ldu, nb, col_base);
+    diag_ul_inv_kernel<T><<<1, DIAG_THREADS, 0, s>>>(A, lda, U, ldu, nb, col_base);
     return launch_status();
 }
 
@@ -125,46 +163,56 @@ __global__ void copy_damped_kernel(const float *H, long long ldh, float *A, long
     }
 }
 
-// Blocked UL factorization + inverse. A (n x n, lda) holds the damped matrix on entry (upper
-// triangle read) and Ubar on exit (upper triangle); U (n x n, ldu) receives the inverse
-// factor (upper; strictly lower part zero). T is scratch of FACTOR_NB x n floats.
+// Recursive UL factorization + inverse of the diagonal block [r0, r1) of A (upper triangle
+// read): A_blk = Ubar Ubar^T, and U[r0:r1, r0:r1] = Ubar^-1 is written. With the block split
+// at m (a multiple of FACTOR_NB) into 1 = [r0, m) and 2 = [m, r1):
+//   U22            <- recursion on block 2 (bottom-right first)
+//   Ubar12 = A12 U22^T             (kept transposed, S12 = U22 A12^T, in A's lower-left block)
+//   A11   -= Ubar12 Ubar12^T       (upper triangle)
+//   U11            <- recursion on block 1
+//   U12 = -U11 (Ubar12 U22)        (the product Ubar12 U22 is staged in A12's place)
+// This is the block form of Ubar U = I. Every step is a large GEMM except the 128-wide leaves
+// (one-CTA diagonal kernel); A's strictly lower triangle is used as scratch, so nothing beyond
+// the n x n work matrix is needed.
+inline int factor_rec(float *A, long long lda, float *U, long long ldu, int r0, int r1,
+                      cudaStream_t s) {
+    const int len = r1 - r0;
+    if (len <= FACTOR_NB)
+        return diag_ul_inv<float>(A + (long long)r0 * lda + r0, lda, U + (long long)r0 * ldu + r0,
+                                  ldu, len, r0, s);
+    const int m = r0 + (ceil_div(len, FACTOR_NB) / 2) * FACTOR_NB;
+    const int n1 = m - r0, n2 = r1 - m;
+    if (int st = factor_rec(A, lda, U, ldu, m, r1, s)) return st;
+    float *A12 = A + (long long)r0 * lda + m;        // n1 x n2
+    float *S12 = A + (long long)m * lda + r0;        // n2 x n1 scratch (below the diagonal)
+    const float *U22 = U + (long long)m * ldu + m;   // n2 x n2 upper
+    // S12 = U22 A12^T
+    auto p2 = gemm_args<float, float>(n2, n1, n2, U22, ldu, 0, A12, lda, 1, S12, lda, 1.f, 0.f);
+    p2.a_upper = 1;
+    if (int st = gemm_f32(p2, s)) return st;
+    // A11 -= S12^T S12 (upper)
+    auto p3 = gemm_args<float, float>(n1, n1, n2, S12, lda, 1, S12, lda, 0,
+                                      A + (long long)r0 * lda + r0, lda, -1.f, 1.f);
+    p3.c_upper = 1;
+    if (int st = gemm_f32(p3, s)) return st;
+    if (int st = factor_rec(A, lda, U, ldu, r0, m, s)) return st;
+    // A12 <- T1 = Ubar12 U22 = S12^T U22
+    auto p5 = gemm_args<float, float>(n1, n2, n2, S12, lda, 1, U22, ldu, 0, A12, lda, 1.f, 0.f);
+    p5.b_upper = 1;
+    if (int st = gemm_f32(p5, s)) return st;
+    // U12 = -U11 T1
+    auto p6 = gemm_args<float, float>(n1, n2, n1, U + (long long)r0 * ldu + r0, ldu, 0, A12, lda, 0,
+                                      U + (long long)r0 * ldu + m, ldu, -1.f, 0.f);
+    p6.a_upper = 1;
+    return gemm_f32(p6, s);
+}
+
+// A (n x n, lda) holds the damped matrix on entry (upper triangle read; the rest of A is
+// scratch); U (n x n, ldu) receives the inverse factor (upper; its strictly lower part must
+// be zero on entry and stays zero).
 inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n,
-                             float *T, cudaStream_t s) {
-    const int P = ceil_div(n, FACTOR_NB);
-    for (int p = P - 1; p >= 0; --p) {
-        const int r0 = p * FACTOR_NB;
-        const int r1 = min(n, r0 + FACTOR_NB);
-        const int nb = r1 - r0;
-        if (int st = diag_ul_inv<float>(A + (long long)r0 * lda + r0, lda,
-                                        U + (long long)r0 * ldu + r0, ldu, nb, r0, s))
-            return st;
-        if (r0 > 0) {
-            // 2. panel: A[0:r0, r0:r1] = A[0:r0, r0:r1] * U_pp^T  (in place: one column tile)
-            auto pa = gemm_args<float, float>(r0, nb, nb, A + r0, lda, 0,
-                                              U + (long long)r0 * ldu + r0, ldu, 1, A + r0, lda,
-                                              1.f, 0.f);
-            if (int st = gemm_simt(pa, s)) return st;
-            // 3. syrk: A[0:r0, 0:r0] -= P P^T (upper)
-            auto ps = gemm_args<float, float>(r0, r0, nb, A + r0, lda, 0, A + r0, lda, 1, A, lda,
-                                              -1.f, 1.f);
-            ps.c_upper = 1;
-            if (int st = gemm_simt(ps, s)) return st;
-        }
-        if (r1 < n) {
-            const int w = n - r1;
-            // 4a. T = Ubar[r0:r1, r1:n] * U[r1:n, r1:n]   (U upper)
-            auto pt = gemm_args<float, float>(nb, w, w, A + (long long)r0 * lda + r1, lda, 0,
-                                              U + (long long)r1 * ldu + r1, ldu, 0, T, n, 1.f, 0.f);
-            pt.b_upper = 1;
-            if (int st = gemm_simt(pt, s)) return st;
-            // 4b. U[r0:r1, r1:n] = -U_pp * T   (U_pp upper)
-            auto pu = gemm_args<float, float>(nb, w, nb, U + (long long)r0 * ldu + r0, ldu, 0, T, n,
-                                              0, U + (long long)r0 * ldu + r1, ldu, -1.f, 0.f);
-            pu.a_upper = 1;
-            if (int st = gemm_simt(pu, s)) return st;
-        }
-    }
-    return GPTQ_OK;
+                             float * /*unused*/, cudaStream_t s) {
+    return factor_rec(A, lda, U, ldu, 0, n, s);
 }
 
 }  // namespace gptq

@@ -22,6 +22,8 @@ struct GemmArgs {
     int c_upper;        // write only C(i,j) with j >= i (tiles strictly below are skipped)
     int a_upper;        // A(i,k) = 0 for k < i (storage there is not read)
     int b_upper;        // B(k,j) = 0 for k > j (storage there is not read)
+    int a_lower;        // A(i,k) = 0 for k > i
+    int b_lower;        // B(k,j) = 0 for k < j
 };
 
 namespace simt {
@@ -46,9 +48,14 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
     int kbeg = 0, kend = p.K;
     if (p.a_upper) kbeg = max(kbeg, i0);
     if (p.b_upper) kend = min(kend, j0 + BN);
+    if (p.a_lower) kend = min(kend, i0 + BM);
+    if (p.b_lower) kbeg = max(kbeg, j0);
     kbeg = (kbeg / BK) * BK;
 
-    for (int k0 = kbeg; k0 < kend; k0 += BK) {
+    // register double buffering: the global loads of K tile k+1 are in flight while tile k
+    // is multiplied out of shared memory
+    float ra[(BM * BK) / NT], rb[(BN * BK) / NT];
+    auto load_tiles = [&](int k0) {
 #pragma unroll
         for (int e = 0; e < (BM * BK) / NT; ++e) {
             const int idx = tid + e * NT;
@@ -56,9 +63,9 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
             if (p.ta) { kk = idx / BM; r = idx % BM; } else { r = idx / BK; kk = idx % BK; }
             const int gi = i0 + r, gk = k0 + kk;
             float v = 0.f;
-            if (gi < p.M && gk < kend && (!p.a_upper || gk >= gi))
+            if (gi < p.M && gk < kend && (!p.a_upper || gk >= gi) && (!p.a_lower || gk <= gi))
                 v = to_f32(p.ta ? p.A[(long long)gk * p.lda + gi] : p.A[(long long)gi * p.lda + gk]);
-            As[kk][r] = v;
+            ra[e] = v;
         }
 #pragma unroll
         for (int e = 0; e < (BN * BK) / NT; ++e) {
@@ -67,23 +74,41 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
             if (p.tb) { c = idx / BK; kk = idx % BK; } else { kk = idx / BN; c = idx % BN; }
             const int gj = j0 + c, gk = k0 + kk;
             float v = 0.f;
-            if (gj < p.N && gk < kend && (!p.b_upper || gk <= gj))
+            if (gj < p.N && gk < kend && (!p.b_upper || gk <= gj) && (!p.b_lower || gk >= gj))
                 v = to_f32(p.tb ? p.B[(long long)gj * p.ldb + gk] : p.B[(long long)gk * p.ldb + gj]);
-            Bs[kk][c] = v;
+            rb[e] = v;
+        }
+    };
+    if (kbeg < kend) load_tiles(kbeg);
+    for (int k0 = kbeg; k0 < kend; k0 += BK) {
+#pragma unroll
+        for (int e = 0; e < (BM * BK) / NT; ++e) {
+            const int idx = tid + e * NT;
+            int r, kk;
+            if (p.ta) { kk = idx / BM; r = idx % BM; } else { r = idx / BK; kk = idx % BK; }
+            As[kk][r] = ra[e];
+        }
+#pragma unroll
+        for (int e = 0; e < (BN * BK) / NT; ++e) {
+            const int idx = tid + e * NT;
+            int c, kk;
+            if (p.tb) { c = idx / BK; kk = idx % BK; } else { kk = idx / BN; c = idx % BN; }
+            Bs[kk][c] = rb[e];
         }
         __syncthreads();
+        if (k0 + BK < kend) load_tiles(k0 + BK);
 #pragma unroll
         for (int kk = 0; kk < BK; ++kk) {
             const float4 a0 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
             const float4 a1 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4 + 64]);
             const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
             const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4 + 64]);
-            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
             for (int i = 0; i < 8; ++i)
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
@@ -119,7 +144,7 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.B = B; p.ldb = ldb; p.tb = tb;
     p.C = C; p.ldc = ldc;
     p.alpha = alpha; p.beta = beta;
-    p.c_upper = 0; p.a_upper = 0; p.b_upper = 0;
+    p.c_upper = 0; p.a_upper = 0; p.b_upper = 0; p.a_lower = 0; p.b_lower = 0;
     return p;
 }
 

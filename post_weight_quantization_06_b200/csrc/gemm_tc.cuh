@@ -1,0 +1,445 @@
+// fp32-accurate GEMM on the tcgen05 tensor cores (kind::tf32, three MMAs per K step):
+//   C = alpha * op(A) op(B) + beta * C          (M x N, fp32 in global memory)
+//
+// The factor and the lazy trailing update need fp32 accuracy: a plain tf32 product moves the
+// pre-rounding values of the sweep by ~1e-3 grid steps. Each fp32 operand x is split into
+// hi = x rounded to the nearest tf32 and lo = (x - hi) rounded to the nearest tf32
+// (|lo| <= 2^-11 |x|); a b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi, error ~2^-22 |a b|.
+//
+// Operand staging: TMA loads 32-deep K slices of both operands with the 128-byte swizzle;
+// "K-major" when K is the contiguous index (one 128-row box), "MN-major" when M / N is (four
+// 32-wide boxes). Converter warps then write lo next to the slice and overwrite the slice
+// with hi (the split is elementwise, so it runs on the swizzled bytes as they are).
+//
+// Warp roles (320 threads, one CTA per SM, persistent over 128 x 128 output tiles):
+//   warp 0     TMA producer, 3-stage ring of {A, A_lo, B, B_lo} (64 KB per stage)
+//   warp 1     TMEM allocation and the MMA issuer (one thread); 3 x 4 MMAs per stage
+//   warps 2-5  hi/lo converters
+//   warps 6-9  epilogue: one row of the tile per thread (TMEM lane = row)
+// Triangular operands: a_upper / a_lower / b_upper / b_lower restrict each tile's K range to
+// where the operand can be nonzero; the storage of the zero triangle must hold zeros.
+// All mbarrier waits are bounded as in the Hessian kernel.
+#pragma once
+
+#include <cuda.h>
+
+#include <cstdlib>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "hessian_tc.cuh"
+
+namespace gptq {
+namespace tcg {
+
+using tc::desc_mn_sw128;
+using tc::mbar_arrive;
+using tc::mbar_expect_tx;
+using tc::mbar_init;
+using tc::mbar_wait;
+using tc::mma_commit;
+using tc::smem_u32;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+using tc::tma_load_2d;
+using tc::tmem_alloc;
+using tc::tmem_dealloc;
+using tc::tmem_relinquish;
+
+constexpr int TILE = 128;
+constexpr int BK = 32;                    // fp32 elements per K slice (128 bytes)
+constexpr int STAGES = 3;
+constexpr int SLICE_BYTES = TILE * BK * 4;          // 16 KB
+constexpr int STAGE_BYTES = 4 * SLICE_BYTES;        // A, A_lo, B, B_lo
+constexpr int CONV_WARPS = 4, EPI_WARPS = 4;
+constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
+constexpr int TMEM_COLS = 2 * TILE;
+constexpr size_t EPI_STAGE_BYTES = (size_t)EPI_WARPS * 32 * 33 * 4;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + EPI_STAGE_BYTES;
+
+__host__ __device__ constexpr uint32_t idesc_tf32(int a_mn, int b_mn) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(TILE >> 3) << 17) | ((uint32_t)(TILE >> 4) << 24);
+}
+
+// K-major operand, 128-byte swizzle: rows of 32 fp32 (128 B), 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t desc_k_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;                         // LBO (unused for swizzled K-major)
+    d |= (uint64_t)((1024 >> 4) & 0x3FFFu) << 32;   // SBO: next 8 rows
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)2 << 61;
+    return d;
+}
+// MN-major operand of tf32: the only MN-major layout the tensor cores take for 32-bit
+// elements is the 128-byte swizzle with 32-byte atoms (layout type 1), whose pattern repeats
+// every 4 K rows. Rows are 128 B (32 M/N elements); 4-row groups are 512 B apart; the 32-wide
+// M/N chunks (one TMA box of BK rows each) are BK * 128 B apart.
+__device__ __forceinline__ uint64_t desc_mn32_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(((BK * 128) >> 4) & 0x3FFFu) << 16;  // LBO: next 32 M/N elements
+    d |= (uint64_t)((512 >> 4) & 0x3FFFu) << 32;         // SBO: next 4 K rows
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)1 << 61;                               // 128B swizzle, 32B atoms
+    return d;
+}
+
+// Round to the nearest tf32 value (kept as an fp32 bit pattern with the low 13 bits zero).
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t dtmem, uint64_t adesc, uint64_t bdesc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(dtmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct TcGemmParams {
+    int M, N, K;
+    float *C;
+    long long ldc;
+    float alpha, beta;
+    int a_mn, b_mn;     // 1: operand is MN-major (M / N contiguous), 0: K-major
+    int c_upper, a_upper, a_lower, b_upper, b_lower;
+    int tiles_m, tiles_n;
+    long long wait_limit;
+};
+
+// K range [kb, ke) (multiples of BK) of output tile (ti, tj).
+__device__ __forceinline__ void tile_k_range(const TcGemmParams &p, int ti, int tj, int &kb,
+                                             int &ke) {
+    int b = 0, e = p.K;
+    const int i0 = ti * TILE, j0 = tj * TILE;
+    if (p.a_upper) b = max(b, i0);
+    if (p.b_lower) b = max(b, j0);
+    if (p.a_lower) e = min(e, i0 + TILE);
+    if (p.b_upper) e = min(e, j0 + TILE);
+    kb = (b / BK) * BK;
+    ke = e;
+}
+
+__device__ __forceinline__ bool tile_skipped(const TcGemmParams &p, int ti, int tj) {
+    return p.c_upper && ti * TILE >= (tj + 1) * TILE;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+               TcGemmParams p) {
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char *base = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + STAGES * STAGE_BYTES);
+    uint64_t *full = bars;                       // TMA -> converters
+    uint64_t *conv = bars + STAGES;              // converters -> MMA
+    uint64_t *empty = bars + 2 * STAGES;         // MMA -> TMA
+    uint64_t *acc_full = bars + 3 * STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *mma_done = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+    float *epi_stage = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = p.tiles_m * p.tiles_n;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&conv[s], CONV_WARPS);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], EPI_WARPS); }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            long long it = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+                const int ti = t / p.tiles_n, tj = t % p.tiles_n;
+                if (tile_skipped(p, ti, tj)) continue;
+                int kb, ke;
+                tile_k_range(p, ti, tj, kb, ke);
+                for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
+                    const int slot = (int)(it % STAGES);
+                    if (*abort_flag) break;
+                    if (!mbar_wait(&empty[slot], (uint32_t)((it / STAGES) & 1) ^ 1u, p.wait_limit)) {
+                        report(GPTQ_ERR_TIMEOUT, 11);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    unsigned char *st = base + slot * STAGE_BYTES;
+                    mbar_expect_tx(&full[slot], 2 * SLICE_BYTES);
+                    if (p.a_mn) {
+                        for (int q = 0; q < 4; ++q)
+                            tma_load_2d(&amap, &full[slot], st + q * (BK * 128), ti * TILE + 32 * q, k0);
+                    } else {
+                        tma_load_2d(&amap, &full[slot], st, k0, ti * TILE);
+                    }
+                    unsigned char *sb = st + 2 * SLICE_BYTES;
+                    if (p.b_mn) {
+                        for (int q = 0; q < 4; ++q)
+                            tma_load_2d(&bmap, &full[slot], sb + q * (BK * 128), tj * TILE + 32 * q, k0);
+                    } else {
+                        tma_load_2d(&bmap, &full[slot], sb, k0, tj * TILE);
+                    }
+                }
+            }
+            if (*abort_flag)
+                for (long long j = it - 1; j >= 0 && j >= it - STAGES; --j)
+                    mbar_wait(&full[j % STAGES], (uint32_t)((j / STAGES) & 1), p.wait_limit);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = idesc_tf32(p.a_mn, p.b_mn);
+            long long it = 0, ch = 0;
+            for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+                const int ti = t / p.tiles_n, tj = t % p.tiles_n;
+                if (tile_skipped(p, ti, tj)) continue;
+                int kb, ke;
+                tile_k_range(p, ti, tj, kb, ke);
+                if (ke <= kb) continue;   // nothing to accumulate: the epilogue writes beta C
+                const int b = (int)(ch & 1);
+                if (!mbar_wait(&acc_empty[b], (uint32_t)((ch >> 1) & 1) ^ 1u, p.wait_limit)) {
+                    report(GPTQ_ERR_TIMEOUT, 12);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dt = tmem + (uint32_t)(b * TILE);
+                for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
+                    const int slot = (int)(it % STAGES);
+                    if (!mbar_wait(&conv[slot], (uint32_t)((it / STAGES) & 1), p.wait_limit)) {
+                        report(GPTQ_ERR_TIMEOUT, 13);
+                        *abort_flag = 1;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(base + slot * STAGE_BYTES);
+                    const uint32_t sal = sa + SLICE_BYTES, sbb = sa + 2 * SLICE_BYTES,
+                                   sbl = sa + 3 * SLICE_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 8; ++kk) {
+                        const uint32_t offa = p.a_mn ? kk * 1024u : kk * 32u;
+                        const uint32_t offb = p.b_mn ? kk * 1024u : kk * 32u;
+                        const uint64_t ah = p.a_mn ? desc_mn32_sw128(sa + offa) : desc_k_sw128(sa + offa);
+                        const uint64_t al = p.a_mn ? desc_mn32_sw128(sal + offa) : desc_k_sw128(sal + offa);
+                        const uint64_t bh = p.b_mn ? desc_mn32_sw128(sbb + offb) : desc_k_sw128(sbb + offb);
+                        const uint64_t bl = p.b_mn ? desc_mn32_sw128(sbl + offb) : desc_k_sw128(sbl + offb);
+                        const uint32_t acc0 = (k0 > kb || kk > 0) ? 1u : 0u;
+                        mma_tf32(dt, ah, bh, idesc, acc0);
+                        mma_tf32(dt, ah, bl, idesc, 1u);
+                        mma_tf32(dt, al, bh, idesc, 1u);
+                    }
+                    mma_commit(&empty[slot]);
+                }
+                mma_commit(&acc_full[b]);
+                ++ch;
+            }
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0, p.wait_limit);
+        }
+    } else if (warp < 2 + CONV_WARPS) {
+        // hi / lo split of each staged slice
+        const int cw = warp - 2;
+        long long it = 0;
+        for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+            const int ti = t / p.tiles_n, tj = t % p.tiles_n;
+            if (tile_skipped(p, ti, tj)) continue;
+            int kb, ke;
+            tile_k_range(p, ti, tj, kb, ke);
+            for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
+                const int slot = (int)(it % STAGES);
+                if (!mbar_wait(&full[slot], (uint32_t)((it / STAGES) & 1), p.wait_limit)) {
+                    if (lane == 0) report(GPTQ_ERR_TIMEOUT, 14);
+                    *abort_flag = 1;
+                    break;
+                }
+                unsigned char *st = base + slot * STAGE_BYTES;
+#pragma unroll
+                for (int op = 0; op < 2; ++op) {
+                    float4 *hi = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES);
+                    float4 *lo = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES + SLICE_BYTES);
+                    for (int i = cw * 32 + lane; i < SLICE_BYTES / 16; i += CONV_WARPS * 32) {
+                        const float4 x = hi[i];
+                        float4 h, l;
+                        h.x = to_tf32(x.x); h.y = to_tf32(x.y); h.z = to_tf32(x.z); h.w = to_tf32(x.w);
+                        l.x = to_tf32(x.x - h.x); l.y = to_tf32(x.y - h.y);
+                        l.z = to_tf32(x.z - h.z); l.w = to_tf32(x.w - h.w);
+                        lo[i] = l;
+                        hi[i] = h;
+                    }
+                }
+                // generic-proxy writes must be visible to the tensor cores' async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&conv[slot]);
+            }
+        }
+    } else {
+        // epilogue: C = alpha * acc + beta * C
+        const int q = warp & 3;
+        long long ch = 0;
+        for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+            const int ti = t / p.tiles_n, tj = t % p.tiles_n;
+            if (tile_skipped(p, ti, tj)) continue;
+            int kb, ke;
+            tile_k_range(p, ti, tj, kb, ke);
+            const bool has_acc = ke > kb;
+            int b = 0;
+            if (has_acc) {
+                b = (int)(ch & 1);
+                if (!mbar_wait(&acc_full[b], (uint32_t)((ch >> 1) & 1), p.wait_limit)) {
+                    if (lane == 0) report(GPTQ_ERR_TIMEOUT, 15);
+                    *abort_flag = 1;
+                    break;
+                }
+                tc_fence_after();
+            }
+            // Each warp owns rows [32 q, 32 q + 32) of the tile. Per 32-column slice the values
+            // (one row per lane) pass through a padded shared buffer so that the global
+            // accesses are whole 128-byte row segments.
+            float *stage = epi_stage + (warp - 2 - CONV_WARPS) * 32 * 33;
+            const int row_base = ti * TILE + 32 * q;
+#pragma unroll 1
+            for (int c32 = 0; c32 < TILE / 32; ++c32) {
+                float v[32];
+                if (has_acc) {
+                    tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * TILE + 32 * c32), v);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
+                __syncwarp();
+                const int col = tj * TILE + 32 * c32 + lane;
+                for (int r = 0; r < 32; ++r) {
+                    const int row = row_base + r;
+                    if (row >= p.M || col >= p.N || (p.c_upper && col < row)) continue;
+                    float *cp = p.C + (long long)row * p.ldc + col;
+                    const float o = p.alpha * stage[r * 33 + lane];
+                    *cp = p.beta == 0.f ? o : fmaf(p.beta, *cp, o);
+                }
+                __syncwarp();
+            }
+            if (has_acc) {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[b]);
+                ++ch;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------------------
+// host side
+// ------------------------------------------------------------------------------------------
+
+// 2D fp32 tensor map over a row-major matrix of `rows` x `cols` (row pitch ld floats) whose
+// contiguous index is `cols`; box = box_cols (contiguous) x box_rows.
+// mn_major selects the 32-byte-atom variant of the 128-byte swizzle that MN-major tf32
+// operands need; K-major operands use the plain 128-byte swizzle.
+inline bool make_map_f32(CUtensorMap *map, const float *ptr, long long rows, long long cols,
+                         long long ld, int box_cols, int box_rows, bool mn_major) {
+    tc::EncodeTiledFn enc = tc::encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)ld * 4};
+    const cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(ptr), dims, strides,
+               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               mn_major ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+           CUDA_SUCCESS;
+}
+
+// True when the tensor-core path can take this product: 16-byte aligned bases and pitches.
+inline bool tc_eligible(const void *A, long long lda, const void *B, long long ldb) {
+    return ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B)) & 15u) == 0 &&
+           lda % 4 == 0 && ldb % 4 == 0;
+}
+
+}  // namespace tcg
+}  // namespace gptq
+
+namespace gptq {
+
+// C = alpha op(A) op(B) + beta C in fp32 accuracy: tcgen05 (tf32 x 3) when the shapes and
+// alignments allow it, the SIMT kernel otherwise (small or unaligned products, or when
+// GPTQ_FORCE_SIMT_GEMM is set).
+inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
+    if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+    const bool small = (long long)g.M * g.N < 128LL * 256 || g.K < 64;
+    if (small || !tcg::tc_eligible(g.A, g.lda, g.B, g.ldb) ||
+        (reinterpret_cast<uintptr_t>(g.C) & 3u) || std::getenv("GPTQ_FORCE_SIMT_GEMM"))
+        return gemm_simt(g, s);
+    tcg::TcGemmParams p;
+    p.M = g.M; p.N = g.N; p.K = g.K;
+    p.C = g.C; p.ldc = g.ldc;
+    p.alpha = g.alpha; p.beta = g.beta;
+    p.a_mn = g.ta ? 1 : 0;
+    p.b_mn = g.tb ? 0 : 1;
+    p.c_upper = g.c_upper; p.a_upper = g.a_upper; p.a_lower = g.a_lower;
+    p.b_upper = g.b_upper; p.b_lower = g.b_lower;
+    p.tiles_m = ceil_div(g.M, tcg::TILE);
+    p.tiles_n = ceil_div(g.N, tcg::TILE);
+    p.wait_limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
+    CUtensorMap am, bm;
+    const bool ok_a = p.a_mn ? tcg::make_map_f32(&am, g.A, g.K, g.M, g.lda, 32, 32, true)
+                             : tcg::make_map_f32(&am, g.A, g.M, g.K, g.lda, 32, tcg::TILE, false);
+    const bool ok_b = p.b_mn ? tcg::make_map_f32(&bm, g.B, g.K, g.N, g.ldb, 32, 32, true)
+                             : tcg::make_map_f32(&bm, g.B, g.N, g.K, g.ldb, 32, tcg::TILE, false);
+    if (!ok_a || !ok_b) return gemm_simt(g, s);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < sms ? tiles : sms;
+    cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tcg::SMEM_BYTES);
+    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, p);
+    return launch_status();
+}
+
+}  // namespace gptq

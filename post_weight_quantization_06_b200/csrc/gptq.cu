@@ -41,10 +41,13 @@ inline FactorWs carve_factor(Carver &c, long long n) {
 struct QuantWs {
     float *Wc, *Err;
 };
+// Err holds the errors of one outer block of the two-level lazy update: m x OB with
+// OB <= min(QUANT_OUTER_MAX, n).
 inline QuantWs carve_quant(Carver &c, long long m, long long N, int B) {
     QuantWs w;
     w.Wc = c.take<float>((size_t)m * N);
-    w.Err = c.take<float>((size_t)m * B);
+    const long long ob = N < QUANT_OUTER_MAX ? N : QUANT_OUTER_MAX;
+    w.Err = c.take<float>((size_t)m * (ob > B ? ob : B));
     return w;
 }
 

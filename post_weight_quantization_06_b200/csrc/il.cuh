@@ -281,7 +281,7 @@ inline int il_factor(const float *H, long long ldh, int n, int r, const float *V
     // U12 = -U11 Yr
     auto p = gemm_args<float, float>(n, r, n, Uaug, ldu, 0, w.Yr, r, 0, Uaug + n, ldu, -1.f, 0.f);
     p.a_upper = 1;
-    return gemm_simt(p, s);
+    return gemm_f32(p, s);
 }
 
 }  // namespace gptq

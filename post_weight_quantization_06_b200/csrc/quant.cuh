@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
 
 namespace gptq {
 
@@ -43,7 +44,8 @@ struct ColloopArgs {
     float *scales;      // m x G
     uint8_t *zeros;     // m x G
     int G;
-    float *err;         // m x B errors of this panel (row stride B)
+    float *err;         // errors of this panel: m x B block at err (row stride lde)
+    long long lde;
     double *loss;       // m or nullptr
 };
 
@@ -73,9 +75,19 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarps = blockDim.x >> 5;
     const int j0 = a.j0;
-    for (int idx = tid; idx < B * B; idx += blockDim.x) {
-        const int t = idx / B, c = idx % B;
-        Us[idx] = a.U[(long long)(j0 + t) * a.ldu + j0 + c];
+    // U block load: eight independent global loads in flight per thread before the stores
+    for (int base = tid; base < B * B; base += 8 * blockDim.x) {
+        float v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = base + u * blockDim.x;
+            v[u] = idx < B * B ? a.U[(long long)(j0 + idx / B) * a.ldu + j0 + idx % B] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int idx = base + u * blockDim.x;
+            if (idx < B * B) Us[idx] = v[u];
+        }
     }
     __syncthreads();
     for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
@@ -195,7 +207,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
         const int row = row0 + r;
 #pragma unroll
         for (int q = 0; q < NSLOT; ++q) {
-            if (rv[r]) a.err[(long long)row * B + 32 * q + lane] = ev[r][q];
+            if (rv[r]) a.err[(long long)row * a.lde + 32 * q + lane] = ev[r][q];
             cb[r * B + 32 * q + lane] = (uint8_t)cv[r][q];
         }
         if (a.loss && lane == 0 && rv[r]) {
@@ -253,31 +265,63 @@ __global__ void extract_R_kernel(const float *Wc, long long ldw, int m, int n, i
 }
 
 // The sweep over all panels of a prepared working copy Wc (m x N, first n columns quantized).
+// Width of the outer blocks of the two-level lazy update: 1024 columns (or n if smaller) when
+// every group that starts inside an outer block also ends inside it, i.e. for one group per
+// row or a group length dividing 1024 (group statistics then see fully updated weights);
+// otherwise one level only (outer width = B). Always <= QUANT_OUTER_MAX, the row stride the
+// workspace reserves for the errors.
+constexpr int QUANT_OUTER_MAX = 1024;
+inline int outer_block(int n, int gs, int B) {
+    const int ob = (gs >= n || QUANT_OUTER_MAX % gs == 0) ? QUANT_OUTER_MAX : B;
+    return ob < n ? ob : n;
+}
+
+// The sweep over all panels of a prepared working copy Wc (m x N, first n columns quantized).
+// Lazy updates are two-level (GPTQ's lazy block update, applied at two widths; GPTQ-2D,
+// Theorem 1: any order that respects the feedback dependencies rounds the same):
+//   after each panel of B columns:      Wc[:, panel_end:outer_end] -= Err_panel U[panel, ...]
+//   after each outer block of OB cols:  Wc[:, outer_end:N]         -= Err_outer U[outer, ...]
+// so the columns far to the right receive one K = OB product per outer block instead of OB/B
+// products with K = B. Err holds m x OB floats.
 inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const float *U,
                        long long ldu, int bits, int group_size, int B, uint32_t *codes,
                        float *scales, uint8_t *zeros, double *loss, float *Err,
                        cudaStream_t s) {
+    const int gs = group_size ? group_size : n;
+    const int OB = outer_block(n, gs, B);
     ColloopArgs a;
     a.Wc = Wc; a.ldw = ldw; a.U = U; a.ldu = ldu; a.m = m; a.n = n;
-    a.bits = bits; a.gs = group_size ? group_size : n;
+    a.bits = bits; a.gs = gs;
     a.codes = codes; a.ldcodes = (long long)n * bits / 32;
     a.scales = scales; a.zeros = zeros; a.G = group_size ? n / group_size : 1;
-    a.err = Err; a.loss = loss;
-    for (int j0 = 0; j0 < n; j0 += B) {
-        a.j0 = j0;
-        int st;
-        switch (B) {
-            case 32: st = colloop_launch<1>(a, s); break;
-            case 64: st = colloop_launch<2>(a, s); break;
-            default: st = colloop_launch<4>(a, s); break;
+    a.lde = OB; a.loss = loss;
+    for (int o0 = 0; o0 < n; o0 += OB) {
+        const int o1 = o0 + OB < n ? o0 + OB : n;
+        for (int j0 = o0; j0 < o1; j0 += B) {
+            a.j0 = j0;
+            a.err = Err + (j0 - o0);
+            int st;
+            switch (B) {
+                case 32: st = colloop_launch<1>(a, s); break;
+                case 64: st = colloop_launch<2>(a, s); break;
+                default: st = colloop_launch<4>(a, s); break;
+            }
+            if (st) return st;
+            const int j1 = j0 + B;
+            if (j1 < o1) {
+                // inner: Wc[:, j1:o1] -= Err_panel (m x B) * U[j0:j1, j1:o1]
+                auto p = gemm_args<float, float>(m, o1 - j1, B, Err + (j0 - o0), OB, 0,
+                                                 U + (long long)j0 * ldu + j1, ldu, 0, Wc + j1,
+                                                 ldw, -1.f, 1.f);
+                if (int st2 = gemm_f32(p, s)) return st2;
+            }
         }
-        if (st) return st;
-        const int j1 = j0 + B;
-        if (j1 < N) {
-            // Wc[:, j1:N] -= Err (m x B) * U[j0:j1, j1:N]
-            auto p = gemm_args<float, float>(m, N - j1, B, Err, B, 0, U + (long long)j0 * ldu + j1,
-                                             ldu, 0, Wc + j1, ldw, -1.f, 1.f);
-            if (int st2 = gemm_simt(p, s)) return st2;
+        if (o1 < N) {
+            // outer: Wc[:, o1:N] -= Err_outer (m x (o1 - o0)) * U[o0:o1, o1:N]
+            auto p = gemm_args<float, float>(m, N - o1, o1 - o0, Err, OB, 0,
+                                             U + (long long)o0 * ldu + o1, ldu, 0, Wc + o1, ldw,
+                                             -1.f, 1.f);
+            if (int st2 = gemm_f32(p, s)) return st2;
         }
     }
     return GPTQ_OK;

@@ -169,6 +169,10 @@ SWEEP_CASES = [
     (50, 256, 3, 64, 64, torch.float32),
     (33, 256, 4, 16, 32, torch.float32),
     (17, 128, 8, 128, 128, torch.float32),
+    # several 1024-column outer blocks of the two-level lazy update
+    (64, 2560, 3, 128, 128, torch.bfloat16),
+    (40, 2048, 4, 0, 128, torch.float32),
+    (24, 3072, 2, 96, 32, torch.float32),
 ]
 
 

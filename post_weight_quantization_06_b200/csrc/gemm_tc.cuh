@@ -143,8 +143,22 @@ __device__ __forceinline__ void tile_k_range(const TcGemmParams &p, int ti, int 
     ke = e;
 }
 
-__device__ __forceinline__ bool tile_skipped(const TcGemmParams &p, int ti, int tj) {
-    return p.c_upper && ti * TILE >= (tj + 1) * TILE;
+// Number of output tiles: with c_upper only the tiles on or above the diagonal exist.
+__host__ __device__ __forceinline__ int num_tiles(const TcGemmParams &p) {
+    return p.c_upper ? p.tiles_n * (p.tiles_n + 1) / 2 : p.tiles_m * p.tiles_n;
+}
+
+// Output tile of linear index t, enumerated so that the tiles with the longest K range come
+// first (the persistent CTAs take tiles round-robin, so equal-work tiles land in the same
+// round): with b_upper the K range of column tile j grows with j, with a_upper it shrinks
+// with the row tile i, and so on; c_upper enumerates the upper triangle row by row.
+__device__ __forceinline__ void tile_of(const TcGemmParams &p, int t, int &ti, int &tj) {
+    if (p.c_upper) { tc::tile_coords(t, p.tiles_n, ti, tj); return; }
+    if (p.b_upper) { tj = p.tiles_n - 1 - t / p.tiles_m; ti = t % p.tiles_m; return; }
+    if (p.b_lower) { tj = t / p.tiles_m; ti = t % p.tiles_m; return; }
+    if (p.a_lower) { ti = p.tiles_m - 1 - t / p.tiles_n; tj = t % p.tiles_n; return; }
+    ti = t / p.tiles_n;
+    tj = t % p.tiles_n;
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -165,7 +179,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     float *epi_stage = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int ntiles = p.tiles_m * p.tiles_n;
+    const int ntiles = num_tiles(p);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
@@ -190,8 +204,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         if (lane == 0) {
             long long it = 0;
             for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
-                const int ti = t / p.tiles_n, tj = t % p.tiles_n;
-                if (tile_skipped(p, ti, tj)) continue;
+                int ti, tj;
+                tile_of(p, t, ti, tj);
                 int kb, ke;
                 tile_k_range(p, ti, tj, kb, ke);
                 for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
@@ -228,8 +242,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             const uint32_t idesc = idesc_tf32(p.a_mn, p.b_mn);
             long long it = 0, ch = 0;
             for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
-                const int ti = t / p.tiles_n, tj = t % p.tiles_n;
-                if (tile_skipped(p, ti, tj)) continue;
+                int ti, tj;
+                tile_of(p, t, ti, tj);
                 int kb, ke;
                 tile_k_range(p, ti, tj, kb, ke);
                 if (ke <= kb) continue;   // nothing to accumulate: the epilogue writes beta C
@@ -278,8 +292,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const int cw = warp - 2;
         long long it = 0;
         for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
-            const int ti = t / p.tiles_n, tj = t % p.tiles_n;
-            if (tile_skipped(p, ti, tj)) continue;
+            int ti, tj;
+            tile_of(p, t, ti, tj);
             int kb, ke;
             tile_k_range(p, ti, tj, kb, ke);
             for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
@@ -315,8 +329,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         const int q = warp & 3;
         long long ch = 0;
         for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
-            const int ti = t / p.tiles_n, tj = t % p.tiles_n;
-            if (tile_skipped(p, ti, tj)) continue;
+            int ti, tj;
+            tile_of(p, t, ti, tj);
             int kb, ke;
             tile_k_range(p, ti, tj, kb, ke);
             const bool has_acc = ke > kb;
@@ -434,7 +448,7 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const int tiles = p.tiles_m * p.tiles_n;
+    const int tiles = tcg::num_tiles(p);
     const int grid = tiles < sms ? tiles : sms;
     cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tcg::SMEM_BYTES);

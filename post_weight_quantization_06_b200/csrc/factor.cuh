@@ -43,8 +43,10 @@ template <typename T>
 __global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, long long lda,
                                                                    T *U, long long ldu, int nb,
                                                                    long long col_base) {
-    __shared__ T colb[2][FACTOR_NB];
-    __shared__ T rowb[2][FACTOR_NB];
+    // wb[c' ] = M[c'][c] for c' < c (column c), -1 at c, M[c][c'] for c' > c (row c); the
+    // pivot M[c][c] separately. Then u_i = ipiv wb[i] (i < c) and v_j = -ipiv wb[j].
+    __shared__ T wb[2][FACTOR_NB];
+    __shared__ T dpiv[2];
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     T M[8][8];
 #pragma unroll
@@ -64,32 +66,37 @@ __global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, l
             if (c >= nb) continue;
             if (tx == cc) {
 #pragma unroll
-                for (int a = 0; a < 8; ++a)
-                    if (ty + 16 * a <= c) colb[buf][ty + 16 * a] = M[a][b];
+                for (int a = 0; a < 8; ++a) {
+                    const int i = ty + 16 * a;
+                    if (i < c) wb[buf][i] = M[a][b];
+                    else if (i == c) { wb[buf][c] = T(-1); dpiv[buf] = M[a][b]; }
+                }
             }
             if (ty == cc) {
 #pragma unroll
                 for (int b2 = 0; b2 < 8; ++b2) {
                     const int j = tx + 16 * b2;
-                    if (j > c && j < nb) rowb[buf][j] = M[b][b2];
+                    if (j > c && j < nb) wb[buf][j] = M[b][b2];
                 }
             }
             __syncthreads();
-            const T d = colb[buf][c];
+            const T d = dpiv[buf];
             const bool bad = !(d > T(0)) || !isfinite((double)d);
             if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
-            const T ipiv = T(1) / (bad ? T(1) : sqrt(d));
+            // 1/sqrt(d): hardware estimate refined by one Newton step
+            const T dd = bad ? T(1) : d;
+            T ipiv = rsqrt(dd);
+            ipiv = ipiv * (T(1.5) - T(0.5) * dd * ipiv * ipiv);
             T u[8], v[8];
 #pragma unroll
             for (int a = 0; a < 8; ++a) {
                 const int i = ty + 16 * a;
-                u[a] = i < c ? colb[buf][i] * ipiv : T(0);
+                u[a] = i < c ? wb[buf][i] * ipiv : T(0);
             }
 #pragma unroll
             for (int b2 = 0; b2 < 8; ++b2) {
                 const int j = tx + 16 * b2;
-                v[b2] = j < c ? -colb[buf][j] * ipiv
-                              : (j == c ? ipiv : (j < nb ? -ipiv * rowb[buf][j] : T(0)));
+                v[b2] = j < nb ? -ipiv * wb[buf][j] : T(0);
             }
             if (tx == cc) {
 #pragma unroll

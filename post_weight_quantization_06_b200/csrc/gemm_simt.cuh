@@ -27,23 +27,27 @@ struct GemmArgs {
 };
 
 namespace simt {
-constexpr int BM = 128, BN = 128, BK = 16, NT = 256;
+constexpr int NT = 256;
 }
 
-template <typename TA, typename TB>
+// BT x BT output tile per CTA of 256 threads (16 x 16), each thread a TM x TM sub-tile made
+// of TM/4 x TM/4 float4 blocks BT/2 apart; BT = 128 for large products, 64 for small ones
+// (four times as many CTAs, a K slice of 32).
+template <typename TA, typename TB, int BT>
 __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
     using namespace simt;
+    constexpr int BM = BT, BN = BT, BK = 2048 / BT, TM = BT / 16, NH = TM / 4;
     const int i0 = blockIdx.y * BM, j0 = blockIdx.x * BN;
     if (p.c_upper && i0 >= j0 + BN) return;
     __shared__ __align__(16) float As[BK][BM + 4];
     __shared__ __align__(16) float Bs[BK][BN + 4];
     const int tid = threadIdx.x;
     const int tx = tid & 15, ty = tid >> 4;
-    float acc[8][8];
+    float acc[TM][TM];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < TM; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+        for (int j = 0; j < TM; ++j) acc[i][j] = 0.f;
 
     int kbeg = 0, kend = p.K;
     if (p.a_upper) kbeg = max(kbeg, i0);
@@ -99,26 +103,28 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
         if (k0 + BK < kend) load_tiles(k0 + BK);
 #pragma unroll
         for (int kk = 0; kk < BK; ++kk) {
-            const float4 a0 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4]);
-            const float4 a1 = *reinterpret_cast<const float4 *>(&As[kk][ty * 4 + 64]);
-            const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4]);
-            const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4 + 64]);
-            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float av[TM], bv[TM];
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
+            for (int h = 0; h < NH; ++h) {
+                const float4 a = *reinterpret_cast<const float4 *>(&As[kk][ty * 4 + h * (BT / 2)]);
+                const float4 b = *reinterpret_cast<const float4 *>(&Bs[kk][tx * 4 + h * (BT / 2)]);
+                av[4 * h] = a.x; av[4 * h + 1] = a.y; av[4 * h + 2] = a.z; av[4 * h + 3] = a.w;
+                bv[4 * h] = b.x; bv[4 * h + 1] = b.y; bv[4 * h + 2] = b.z; bv[4 * h + 3] = b.w;
+            }
 #pragma unroll
-                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+            for (int i = 0; i < TM; ++i)
+#pragma unroll
+                for (int j = 0; j < TM; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
         }
         __syncthreads();
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int gi = i0 + ty * 4 + (i & 3) + (i >> 2) * 64;
+    for (int i = 0; i < TM; ++i) {
+        const int gi = i0 + ty * 4 + (i & 3) + (i >> 2) * (BT / 2);
         if (gi >= p.M) continue;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int gj = j0 + tx * 4 + (j & 3) + (j >> 2) * 64;
+        for (int j = 0; j < TM; ++j) {
+            const int gj = j0 + tx * 4 + (j & 3) + (j >> 2) * (BT / 2);
             if (gj >= p.N || (p.c_upper && gj < gi)) continue;
             float *c = p.C + (long long)gi * p.ldc + gj;
             *c = p.beta == 0.f ? p.alpha * acc[i][j] : fmaf(p.alpha, acc[i][j], p.beta * *c);
@@ -129,8 +135,14 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
 template <typename TA, typename TB>
 inline int gemm_simt(const GemmArgs<TA, TB> &p, cudaStream_t s) {
     if (p.M <= 0 || p.N <= 0) return GPTQ_OK;
-    dim3 grid(ceil_div(p.N, simt::BN), ceil_div(p.M, simt::BM));
-    gemm_simt_kernel<TA, TB><<<grid, simt::NT, 0, s>>>(p);
+    // fewer than ~one 128-tile wave: use 64 x 64 tiles for four times the CTAs
+    if ((long long)ceil_div(p.M, 128) * ceil_div(p.N, 128) < 148) {
+        dim3 grid(ceil_div(p.N, 64), ceil_div(p.M, 64));
+        gemm_simt_kernel<TA, TB, 64><<<grid, simt::NT, 0, s>>>(p);
+    } else {
+        dim3 grid(ceil_div(p.N, 128), ceil_div(p.M, 128));
+        gemm_simt_kernel<TA, TB, 128><<<grid, simt::NT, 0, s>>>(p);
+    }
     return launch_status();
 }
 

@@ -208,6 +208,24 @@ def hessian_flops(layer) -> float:
     return float(layer.k) * layer.n * (layer.n + 1)
 
 
+def hessian_traffic(layer):
+    """DRAM bytes per Hessian launch from the committed ncu summary, for the full 2048x6144 /
+    262144-token workload only, and only while the kernel source is the one profiled."""
+    import hashlib
+    import re
+    if (layer.n, layer.k) != (6144, 262144):
+        return None
+    try:
+        txt = open(os.path.join(ROOT, "profiles", "hessian_tc.md")).read()
+        traffic = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt).group(1))
+        src = re.search(r"kernel_source:\s*(\S+)", txt).group(1)
+        digest = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt).group(1)
+        current = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
+    except (OSError, AttributeError, ValueError):
+        return None
+    return traffic if current == digest else None
+
+
 def run_e2e(g, layer, lp, steps, warmup, chunk_tokens=32768):
     """Same pass, inputs from pinned host memory: per step the calibration chunks and W are
     copied host -> device (copies of chunk i+1 overlap the Hessian of chunk i on a second
@@ -395,7 +413,8 @@ def bench_ours(args):
             "roofline": {"bound": "tensor", "kernel": "hessian (2 X^T X)",
                          "achieved": h_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": h_tflops / peak, "peak_source": peak_src,
-                         "traffic": None},
+                         "traffic": hessian_traffic(layer),
+                         "traffic_unit": "bytes per launch (DRAM read + write)"},
             "gpu_launches": int(launches),
             "clocks": clk,
             "device_status": int(st),

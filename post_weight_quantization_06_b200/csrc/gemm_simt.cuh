@@ -118,6 +118,26 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
         }
         __syncthreads();
     }
+    // epilogue: with beta != 0 every read of C is issued before the first write (one round
+    // trip instead of one per element)
+    if (p.beta != 0.f) {
+#pragma unroll
+        for (int i = 0; i < TM; ++i) {
+            const int gi = i0 + ty * 4 + (i & 3) + (i >> 2) * (BT / 2);
+#pragma unroll
+            for (int j = 0; j < TM; ++j) {
+                const int gj = j0 + tx * 4 + (j & 3) + (j >> 2) * (BT / 2);
+                const bool ok = gi < p.M && gj < p.N && !(p.c_upper && gj < gi);
+                acc[i][j] = p.alpha * acc[i][j] +
+                            (ok ? p.beta * p.C[(long long)gi * p.ldc + gj] : 0.f);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < TM; ++i)
+#pragma unroll
+            for (int j = 0; j < TM; ++j) acc[i][j] *= p.alpha;
+    }
 #pragma unroll
     for (int i = 0; i < TM; ++i) {
         const int gi = i0 + ty * 4 + (i & 3) + (i >> 2) * (BT / 2);
@@ -126,8 +146,7 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
         for (int j = 0; j < TM; ++j) {
             const int gj = j0 + tx * 4 + (j & 3) + (j >> 2) * (BT / 2);
             if (gj >= p.N || (p.c_upper && gj < gi)) continue;
-            float *c = p.C + (long long)gi * p.ldc + gj;
-            *c = p.beta == 0.f ? p.alpha * acc[i][j] : fmaf(p.alpha, acc[i][j], p.beta * *c);
+            p.C[(long long)gi * p.ldc + gj] = acc[i][j];
         }
     }
 }

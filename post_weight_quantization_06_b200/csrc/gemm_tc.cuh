@@ -362,12 +362,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
                 __syncwarp();
                 const int col = tj * TILE + 32 * c32 + lane;
+                // all 32 reads of C are issued before any write (the compiler cannot reorder
+                // them across the stores itself), so the read-modify-write costs one round trip
+                float cin[32];
+                if (p.beta != 0.f) {
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) {
+                        const int row = row_base + r;
+                        const bool ok = row < p.M && col < p.N && !(p.c_upper && col < row);
+                        cin[r] = ok ? p.C[(long long)row * p.ldc + col] : 0.f;
+                    }
+                }
+#pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     const int row = row_base + r;
                     if (row >= p.M || col >= p.N || (p.c_upper && col < row)) continue;
-                    float *cp = p.C + (long long)row * p.ldc + col;
                     const float o = p.alpha * stage[r * 33 + lane];
-                    *cp = p.beta == 0.f ? o : fmaf(p.beta, *cp, o);
+                    p.C[(long long)row * p.ldc + col] = p.beta == 0.f ? o : fmaf(p.beta, cin[r], o);
                 }
                 __syncwarp();
             }

@@ -8,10 +8,13 @@
 // Then U^T U = Ubar^-T Ubar^-1 = A^-1, and since the upper factor of A^-1 with a positive
 // diagonal is unique, this is the U of the chol -> inverse -> chol route.
 //
-// Recursive, bottom-right half first (factor_rec below): the work is four large GEMMs per
-// split (tensor cores through gemm_f32) and one-CTA register-tiled kernels on the
-// 128-column diagonal leaves (diag_ul_inv_kernel).
+// Blocked and right-looking, last block first (factor_ul_inverse below): a chain of
+// one-CTA leaf kernels and small panel GEMMs on a high-priority stream, with the trailing
+// updates and the rows of the inverse as tensor-core GEMMs on two more streams.
 #pragma once
+
+#include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "gemm_simt.cuh"
@@ -170,56 +173,305 @@ __global__ void copy_damped_kernel(const float *H, long long ldh, float *A, long
     }
 }
 
-// Recursive UL factorization + inverse of the diagonal block [r0, r1) of A (upper triangle
-// read): A_blk = Ubar Ubar^T, and U[r0:r1, r0:r1] = Ubar^-1 is written. With the block split
-// at m (a multiple of FACTOR_NB) into 1 = [r0, m) and 2 = [m, r1):
-//   U22            <- recursion on block 2 (bottom-right first)
-//   Ubar12 = A12 U22^T             (kept transposed, S12 = U22 A12^T, in A's lower-left block)
-//   A11   -= Ubar12 Ubar12^T       (upper triangle)
-//   U11            <- recursion on block 1
-//   U12 = -U11 (Ubar12 U22)        (the product Ubar12 U22 is staged in A12's place)
-// This is the block form of Ubar U = I. Every step is a large GEMM except the 128-wide leaves
-// (one-CTA diagonal kernel); A's strictly lower triangle is used as scratch, so nothing beyond
-// the n x n work matrix is needed.
-inline int factor_rec(float *A, long long lda, float *U, long long ldu, int r0, int r1,
-                      cudaStream_t s) {
-    const int len = r1 - r0;
-    if (len <= FACTOR_NB)
-        return diag_ul_inv<float>(A + (long long)r0 * lda + r0, lda, U + (long long)r0 * ldu + r0,
-                                  ldu, len, r0, s);
-    const int m = r0 + (ceil_div(len, FACTOR_NB) / 2) * FACTOR_NB;
-    const int n1 = m - r0, n2 = r1 - m;
-    if (int st = factor_rec(A, lda, U, ldu, m, r1, s)) return st;
-    float *A12 = A + (long long)r0 * lda + m;        // n1 x n2
-    float *S12 = A + (long long)m * lda + r0;        // n2 x n1 scratch (below the diagonal)
-    const float *U22 = U + (long long)m * ldu + m;   // n2 x n2 upper
-    // S12 = U22 A12^T
-    auto p2 = gemm_args<float, float>(n2, n1, n2, U22, ldu, 0, A12, lda, 1, S12, lda, 1.f, 0.f);
-    p2.a_upper = 1;
-    if (int st = gemm_f32(p2, s)) return st;
-    // A11 -= S12^T S12 (upper)
-    auto p3 = gemm_args<float, float>(n1, n1, n2, S12, lda, 1, S12, lda, 0,
-                                      A + (long long)r0 * lda + r0, lda, -1.f, 1.f);
-    p3.c_upper = 1;
-    if (int st = gemm_f32(p3, s)) return st;
-    if (int st = factor_rec(A, lda, U, ldu, r0, m, s)) return st;
-    // A12 <- T1 = Ubar12 U22 = S12^T U22
-    auto p5 = gemm_args<float, float>(n1, n2, n2, S12, lda, 1, U22, ldu, 0, A12, lda, 1.f, 0.f);
-    p5.b_upper = 1;
-    if (int st = gemm_f32(p5, s)) return st;
-    // U12 = -U11 T1
-    auto p6 = gemm_args<float, float>(n1, n2, n1, U + (long long)r0 * ldu + r0, ldu, 0, A12, lda, 0,
-                                      U + (long long)r0 * ldu + m, ldu, -1.f, 0.f);
-    p6.a_upper = 1;
-    return gemm_f32(p6, s);
+// ---------------------------------------------------------------------------------------
+// Leaf of the blocked factor (fp32): the same UL sweep as diag_ul_inv_kernel, organised so
+// that no step waits on a CTA-wide barrier. Warp w owns the 16 columns 16w..16w+15; lane l
+// holds rows l, l+32, l+64, l+96 of them (64 registers). Step c belongs to the warp that
+// owns column c: it takes the pivot, publishes u = M[:c, c] / sqrt(d) and 1/sqrt(d) to
+// shared memory (one slot per step, written once) and its 32 lanes arrive on the step's
+// mbarrier (release). Every other warp waits on that barrier (acquire; the hardware parks
+// the waiting threads) and applies the step to its own columns: the Cholesky update
+// (v_j = -u_j) left of c, the inverse update (v_j = -P[c][j] / sqrt(d), row c read from the
+// lane that holds it) right of c.
+//   Row c is final after step c (row c of the inverse, columns >= c): it goes to shared
+// memory and its registers are dead, as are all rows below it, so step c only touches the
+// row slots that still hold rows < c. During its 16 steps the owner rotates its columns by
+// one register position per step (the update of position p lands in p + 1, the restarted
+// pivot column in 0), so the pivot is always in position 15 and every register index is a
+// compile-time constant; 16 rotations restore the order. Only the loop over the 4 row slots
+// is unrolled, which keeps the code each warp runs within the instruction cache.
+// ---------------------------------------------------------------------------------------
+constexpr int LEAF_THREADS = 256;
+constexpr int LEAF_LD = FACTOR_NB + 1;  // padded stride of the staging tile
+constexpr size_t LEAF_SMEM = sizeof(float) * (2 * (size_t)FACTOR_NB * FACTOR_NB + FACTOR_NB);
+static_assert(FACTOR_NB * LEAF_LD <= 2 * FACTOR_NB * FACTOR_NB, "staging fits the step slots");
+
+template <int RC>
+__device__ __forceinline__ void leaf_rotate(float (&M)[4][16]) {
+#pragma unroll
+    for (int r = 0; r <= RC; ++r) {
+        const float t = M[r][15];
+#pragma unroll
+        for (int p = 14; p >= 0; --p) M[r][p + 1] = M[r][p];
+        M[r][0] = t;
+    }
 }
 
-// A (n x n, lda) holds the damped matrix on entry (upper triangle read; the rest of A is
-// scratch); U (n x n, ldu) receives the inverse factor (upper; its strictly lower part must
-// be zero on entry and stays zero).
-inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n,
-                             float * /*unused*/, cudaStream_t s) {
-    return factor_rec(A, lda, U, ldu, 0, n, s);
+// Steps c = 32 RC + 31 .. 32 RC of the sweep (rows of slot RC).
+template <int RC>
+__device__ __forceinline__ void leaf_slot_steps(float (&M)[4][16], float *pub, float *xrow,
+                                                float *pipiv, uint64_t *step_bar, int nb,
+                                                long long col_base, long long wait_limit,
+                                                int lane, int w, bool &stop) {
+#pragma unroll 1
+    for (int cc = 31; cc >= 0; --cc) {
+        const int c = 32 * RC + cc, ob = c >> 4, s = 15 - (c & 15);
+        if (stop) return;
+        if (c >= nb) {
+            if (w == ob) leaf_rotate<RC>(M);  // keep the owner's rotation count
+            continue;
+        }
+        float u[RC + 1], v[16];
+        if (w == ob) {
+            const float d = __shfl_sync(0xffffffffu, M[RC][15], cc);
+            const bool bad = !(d > 0.f) || !isfinite(d);
+            if (bad && lane == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
+            const float dd = bad ? 1.f : d;
+            float ipiv = rsqrtf(dd);
+            ipiv = ipiv * (1.5f - 0.5f * dd * ipiv * ipiv);  // one Newton step
+#pragma unroll
+            for (int r = 0; r <= RC; ++r) {
+                u[r] = (r < RC || lane < cc) ? M[r][15] * ipiv : 0.f;
+                pub[c * FACTOR_NB + lane + 32 * r] = u[r];
+            }
+            if (lane == 0) pipiv[c] = ipiv;
+            tc::mbar_arrive(&step_bar[c]);
+            // position p holds column 16 ob + ((p - s) mod 16): p < s right of c, s <= p < 15
+            // left of c (its u sits in lane (16 ob + p - s) mod 32 of this slot)
+            const int jl = (16 * ob - s) & 31;
+#pragma unroll
+            for (int p = 0; p < 15; ++p) {
+                const float a = __shfl_sync(0xffffffffu, M[RC][p], cc);
+                const float b = __shfl_sync(0xffffffffu, u[RC], (jl + p) & 31);
+                v[p] = p < s ? -ipiv * a : -b;
+            }
+            v[15] = ipiv;
+            if (lane == cc) {
+#pragma unroll
+                for (int p = 0; p < 16; ++p)
+                    if (p < s || p == 15) xrow[c * FACTOR_NB + 16 * ob + ((p - s) & 15)] = v[p];
+            }
+#pragma unroll
+            for (int r = 0; r <= RC; ++r) {
+#pragma unroll
+                for (int p = 14; p >= 0; --p) M[r][p + 1] = fmaf(u[r], v[p], M[r][p]);
+                M[r][0] = u[r] * ipiv;
+            }
+        } else {
+            if (!tc::mbar_wait(&step_bar[c], 0u, wait_limit)) {
+                if (lane == 0) report(GPTQ_ERR_TIMEOUT, col_base + c);
+                stop = true;
+                return;
+            }
+            const float ipiv = pipiv[c];
+#pragma unroll
+            for (int r = 0; r <= RC; ++r) u[r] = pub[c * FACTOR_NB + lane + 32 * r];
+            if (w < ob) {
+                const float4 *q = reinterpret_cast<const float4 *>(pub + c * FACTOR_NB + 16 * w);
+#pragma unroll
+                for (int b4 = 0; b4 < 4; ++b4) {
+                    const float4 x = q[b4];
+                    v[4 * b4 + 0] = -x.x; v[4 * b4 + 1] = -x.y;
+                    v[4 * b4 + 2] = -x.z; v[4 * b4 + 3] = -x.w;
+                }
+            } else {
+#pragma unroll
+                for (int b = 0; b < 16; ++b) v[b] = -ipiv * __shfl_sync(0xffffffffu, M[RC][b], cc);
+                if (lane == cc) {
+                    float4 *q = reinterpret_cast<float4 *>(xrow + c * FACTOR_NB + 16 * w);
+#pragma unroll
+                    for (int b4 = 0; b4 < 4; ++b4)
+                        q[b4] = make_float4(v[4 * b4], v[4 * b4 + 1], v[4 * b4 + 2], v[4 * b4 + 3]);
+                }
+            }
+#pragma unroll
+            for (int r = 0; r <= RC; ++r)
+#pragma unroll
+                for (int b = 0; b < 16; ++b) M[r][b] = fmaf(u[r], v[b], M[r][b]);
+        }
+    }
+}
+
+__global__ __launch_bounds__(LEAF_THREADS) void leaf_ul_inv_kernel(const float *A, long long lda,
+                                                                   float *U, long long ldu, int nb,
+                                                                   long long col_base,
+                                                                   long long wait_limit) {
+    extern __shared__ __align__(16) float leaf_sm[];
+    float *stage = leaf_sm;                              // [128][LEAF_LD], before the sweep
+    float *pub = leaf_sm;                                // [128][128]: u of step c at pub[128 c]
+    float *xrow = leaf_sm + FACTOR_NB * FACTOR_NB;       // [128][128]: rows of the inverse
+    float *pipiv = leaf_sm + 2 * FACTOR_NB * FACTOR_NB;  // [128]
+    __shared__ uint64_t step_bar[FACTOR_NB];             // one single-use barrier per step
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+
+    // stage the block symmetrically from its upper triangle (coalesced rows)
+#pragma unroll 8
+    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
+        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
+        const float v = (j >= i && i < nb && j < nb) ? A[(long long)i * lda + j] : 0.f;
+        if (j >= i) {
+            stage[i * LEAF_LD + j] = v;
+            stage[j * LEAF_LD + i] = v;
+        }
+    }
+    if (tid < FACTOR_NB) tc::mbar_init(&step_bar[tid], 32);
+    __syncthreads();
+    float M[4][16];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int b = 0; b < 16; ++b) M[r][b] = stage[(lane + 32 * r) * LEAF_LD + 16 * w + b];
+    __syncthreads();
+
+    bool stop = false;
+    leaf_slot_steps<3>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
+                       stop);
+    leaf_slot_steps<2>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
+                       stop);
+    leaf_slot_steps<1>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
+                       stop);
+    leaf_slot_steps<0>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
+                       stop);
+    __syncthreads();
+#pragma unroll 8
+    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
+        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
+        if (i < nb && j < nb) U[(long long)i * ldu + j] = j >= i ? xrow[i * FACTOR_NB + j] : 0.f;
+    }
+}
+
+inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, int nb,
+                       long long col_base, cudaStream_t s) {
+    // GPTQ_WARP_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
+    static const bool warp_leaf = tc::env_ll("GPTQ_WARP_LEAF", 1) != 0;
+    if (!warp_leaf) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
+    cudaFuncSetAttribute(leaf_ul_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)LEAF_SMEM);
+    // clock cycles a warp waits for a step before the kernel gives up with GPTQ_ERR_TIMEOUT
+    static const long long limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
+    leaf_ul_inv_kernel<<<1, LEAF_THREADS, LEAF_SMEM, s>>>(A, lda, U, ldu, nb, col_base, limit);
+    return launch_status();
+}
+
+// Streams of the blocked factor: the pivot chain (leaf, panel solve, look-ahead column) on a
+// high-priority stream, the trailing update and the inverse's rows on two others. One set per
+// device, made on the first call; the mutex keeps the event protocol of one call intact
+// against calls from other host threads.
+struct FactorStreams {
+    cudaStream_t chain = nullptr, bulk = nullptr, inv = nullptr;
+    cudaEvent_t fork = nullptr, panel = nullptr, bulk_done = nullptr, join[3] = {};
+    std::mutex mu;
+    bool ready = false;
+};
+
+inline FactorStreams *factor_streams() {
+    static FactorStreams fs[64];
+    static std::mutex init_mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(init_mu);
+    FactorStreams &f = fs[dev];
+    if (!f.ready) {
+        int lo = 0, hi = 0;
+        cudaDeviceGetStreamPriorityRange(&lo, &hi);
+        bool ok = cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, hi) == cudaSuccess &&
+                  cudaStreamCreateWithPriority(&f.bulk, cudaStreamNonBlocking, lo) == cudaSuccess &&
+                  cudaStreamCreateWithPriority(&f.inv, cudaStreamNonBlocking, lo) == cudaSuccess;
+        cudaEvent_t *evs[] = {&f.fork, &f.panel, &f.bulk_done, &f.join[0], &f.join[1], &f.join[2]};
+        for (cudaEvent_t *e : evs)
+            ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return nullptr;
+        f.ready = true;
+    }
+    return &f;
+}
+
+// Blocked right-looking UL factor with the inverse formed alongside (fp32, tensor-core
+// GEMMs). A (n x n, lda) holds the damped matrix in its upper triangle on entry; its strictly
+// lower block rows receive the panels transposed and the upper triangle is consumed. U (n x
+// n, ldu) must be zero on entry and receives U = Ubar^-1, where A = Ubar Ubar^T, Ubar upper
+// (so that A^-1 = U^T U with U upper: the factor the column sweep uses). With 128-column
+// blocks k = K-1 .. 0, r = first column of block k:
+//   chain  X_kk  = leaf(A_kk)                              (Ubar_kk^-1)
+//          L_k^T = X_kk A[0:r, k]^T                         (panel of Ubar, kept transposed)
+//          A[0:r, k-1] -= L_k L_k[k-1]^T                    (look-ahead: the next panel)
+//   bulk   A[0:r', 0:r'] -= L_k L_k^T on r' = start of block k-1 (upper triangle)
+//   inv    U[k, >k] = -X_kk P[k, >k],  P[0:r, k:] += L_k U[k, k:]
+// where P = U's upper part before its row block is final: P[i, j] = sum_l Ubar[i, l] X[l, j]
+// over the finished row blocks l, from Ubar X = I. The chain waits for the bulk update of
+// the previous block before its look-ahead; the inverse stream trails both.
+inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n, float *T,
+                             cudaStream_t s) {
+    if (n <= FACTOR_NB) return leaf_ul_inv(A, lda, U, ldu, n, 0, s);
+    FactorStreams *fs = factor_streams();
+    if (!fs) return GPTQ_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(fs->mu);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // persistent CTAs of each side-stream GEMM: the rest of the SMs stay free for the chain
+    static const long long side_env = tc::env_ll("GPTQ_FACTOR_SIDE_CTAS", 0);
+    const int side = side_env > 0 ? (int)side_env : (2 * sms) / 3;
+    if (cudaEventRecord(fs->fork, s) != cudaSuccess) return GPTQ_ERR_CUDA;
+    cudaStreamWaitEvent(fs->chain, fs->fork, 0);
+    cudaStreamWaitEvent(fs->bulk, fs->fork, 0);
+    cudaStreamWaitEvent(fs->inv, fs->fork, 0);
+    const int K = ceil_div(n, FACTOR_NB);
+    int st = GPTQ_OK;
+    for (int k = K - 1; k >= 0 && st == GPTQ_OK; --k) {
+        const int r = k * FACTOR_NB, bk = std::min(FACTOR_NB, n - r);
+        float *Xkk = U + (long long)r * ldu + r;
+        float *Lt = A + (long long)r * lda;  // L_k^T: bk x r, strict lower block row k
+        if ((st = leaf_ul_inv(A + (long long)r * lda + r, lda, Xkk, ldu, bk, r, fs->chain))) break;
+        if (k > 0) {
+            auto p = gemm_args<float, float>(bk, r, bk, Xkk, ldu, 0, A + r, lda, 1, Lt, lda, 1.f, 0.f);
+            p.a_upper = 1;
+            if ((st = gemm_f32(p, fs->chain))) break;
+        }
+        cudaEventRecord(fs->panel, fs->chain);
+        if (k > 0) {
+            const int r1 = r - FACTOR_NB;
+            cudaStreamWaitEvent(fs->chain, fs->bulk_done, 0);  // bulk update of block k+1
+            auto p = gemm_args<float, float>(r, FACTOR_NB, bk, Lt, lda, 1, Lt + r1, lda, 0, A + r1,
+                                             lda, -1.f, 1.f);
+            if ((st = gemm_f32(p, fs->chain))) break;
+            if (r1 > 0) {
+                cudaStreamWaitEvent(fs->bulk, fs->panel, 0);
+                auto q = gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);
+                q.c_upper = 1;
+                q.max_ctas = side;
+                if ((st = gemm_f32(q, fs->bulk))) break;
+                cudaEventRecord(fs->bulk_done, fs->bulk);
+            }
+        }
+        cudaStreamWaitEvent(fs->inv, fs->panel, 0);
+        if (k < K - 1) {
+            const int e = r + bk, wdt = n - e;
+            float *row = U + (long long)r * ldu + e;
+            if (cudaMemcpy2DAsync(T, sizeof(float) * wdt, row, sizeof(float) * ldu,
+                                  sizeof(float) * wdt, bk, cudaMemcpyDeviceToDevice,
+                                  fs->inv) != cudaSuccess) {
+                st = GPTQ_ERR_CUDA;
+                break;
+            }
+            auto p = gemm_args<float, float>(bk, wdt, bk, Xkk, ldu, 0, T, wdt, 0, row, ldu, -1.f, 0.f);
+            p.a_upper = 1;
+            p.max_ctas = side;
+            if ((st = gemm_f32(p, fs->inv))) break;
+        }
+        if (k > 0) {
+            auto p = gemm_args<float, float>(r, n - r, bk, Lt, lda, 1, Xkk, ldu, 0, U + r, ldu, 1.f, 1.f);
+            p.max_ctas = side;
+            if ((st = gemm_f32(p, fs->inv))) break;
+        }
+    }
+    // join all three streams back into the caller's stream, on success and on error alike
+    cudaEventRecord(fs->join[0], fs->chain);
+    cudaEventRecord(fs->join[1], fs->bulk);
+    cudaEventRecord(fs->join[2], fs->inv);
+    for (int i = 0; i < 3; ++i) cudaStreamWaitEvent(s, fs->join[i], 0);
+    if (st == GPTQ_OK && cudaGetLastError() != cudaSuccess) st = GPTQ_ERR_CUDA;
+    return st;
 }
 
 }  // namespace gptq

@@ -24,6 +24,8 @@ struct GemmArgs {
     int b_upper;        // B(k,j) = 0 for k > j (storage there is not read)
     int a_lower;        // A(i,k) = 0 for k > i
     int b_lower;        // B(k,j) = 0 for k < j
+    int max_ctas;       // > 0: at most this many persistent CTAs (tensor-core path only), so
+                        // that kernels on other streams keep SMs
 };
 
 namespace simt {
@@ -176,6 +178,7 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.C = C; p.ldc = ldc;
     p.alpha = alpha; p.beta = beta;
     p.c_upper = 0; p.a_upper = 0; p.b_upper = 0; p.a_lower = 0; p.b_lower = 0;
+    p.max_ctas = 0;
     return p;
 }
 

@@ -460,7 +460,8 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int tiles = tcg::num_tiles(p);
-    const int grid = tiles < sms ? tiles : sms;
+    int grid = tiles < sms ? tiles : sms;
+    if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
     cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tcg::SMEM_BYTES);
     tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, p);

@@ -227,7 +227,10 @@ GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64
         // tensor-core path: TMA needs a 16-byte aligned base and 16-byte row pitch
         if (n % 8 == 0 && (reinterpret_cast<uintptr_t>(X) & 15u) == 0 &&
             std::getenv("GPTQ_FORCE_SIMT_HESSIAN") == nullptr)
-            return tc::hessian_tc(H, Xb, k, (int)n, s);
+        {
+            if (int st = tc::hessian_tc(H, Xb, k, (int)n, s)) return st;
+            return mirror_upper(H, n, n, s);
+        }
         return hessian_simt(H, Xb, k, (int)n, s);
     }
     return hessian_simt(H, static_cast<const float *>(X), k, (int)n, s);

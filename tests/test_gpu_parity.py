@@ -66,7 +66,7 @@ def test_hessian_bf16(g, n, k, chunks):
 
 @pytest.mark.parametrize("n,k", [(512, 20000), (1536, 65536)])
 def test_hessian_tensor_core_path_is_tighter_than_fp32_chain(g, n, k, monkeypatch):
-    """bf16 X with n % 8 == 0 runs on tcgen05 with compensated chunk sums; the SIMT path
+    """bf16 X with n % 8 == 0 runs on tcgen05 with two-level chunk sums; the SIMT path
     (forced by GPTQ_FORCE_SIMT_HESSIAN) is a plain fp32 chain. Both against the oracle."""
     X = torch.from_numpy(_spd_from_data(n, k, 3 * n)).float().to(DEV).to(torch.bfloat16)
     Href = oracle.hessian(np64(X))
@@ -93,7 +93,7 @@ def test_hessian_bounded_wait_reports_timeout_and_device_stays_usable(g, monkeyp
     H = torch.zeros(n, n, device=DEV)
     g.gptq_hessian_accumulate(H, X)
     st, info = g.gptq_sync_status(raise_on_error=False)
-    assert st == g.GPTQ_ERR_TIMEOUT and info in (1, 2, 3, 4, 5)
+    assert st == g.GPTQ_ERR_TIMEOUT and info in (1, 2, 3, 4, 5, 6, 7)
     monkeypatch.delenv("GPTQ_TEST_STALL")
     monkeypatch.delenv("GPTQ_WAIT_LIMIT_CYCLES")
     H.zero_()

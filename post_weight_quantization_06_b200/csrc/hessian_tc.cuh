@@ -61,7 +61,16 @@ constexpr int STAGE_BYTES = 2 * HALF_BYTES;  // this CTA's halves of A and B
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr int TMEM_COLS = 2 * PAIR_TILE;     // two 128-lane x 256-column accumulators
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256;
+// Each epilogue thread sums 128 columns of its TMEM lane: the first ACC_REGS in registers,
+// the rest in shared memory (column-major over the 256 epilogue threads), which keeps the
+// kernel within the 168 registers a thread can have with 10 warps per SM and off the
+// local-memory spill path.
+constexpr int ACC_REGS = 96;
+constexpr int ACC_SMEM = 128 - ACC_REGS;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
+constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 +
+                              sizeof(float) * (size_t)ACC_SMEM * EPI_THREADS;
+static_assert(SMEM_BYTES <= 232448, "fits the 227 KB of shared memory a CTA may use");
 
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both MN-major, M = N = 256 (the
 // pair's shape: each CTA supplies 128 rows of A and 128 columns of B and receives 128 rows
@@ -427,7 +436,9 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HessianParams p) {
         const int e = warp - 2;
         const int q = warp & 3;         // TMEM lane quarter this warp may access
         const int h = e >> 2;           // column half
-        float acc[128];
+        float acc[ACC_REGS];
+        float *acc_sm = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) +
+                        (threadIdx.x - 64);  // column j at acc_sm[j * EPI_THREADS]
         int ch = 0;
         if (p.stall) {
             if (!mbar_wait(never, 0, p.wait_limit)) {
@@ -435,13 +446,16 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HessianParams p) {
                 *abort_flag = 1;
             }
         }
+        // running sum of column c of this thread (c compile-time after unrolling)
+#define HESS_ACC(c) (*((c) < ACC_REGS ? &acc[(c) < ACC_REGS ? (c) : 0] \
+                                       : &acc_sm[((c) < ACC_REGS ? 0 : (c) - ACC_REGS) * EPI_THREADS]))
         const uint32_t tq = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(128 * h);
         const uint32_t rel0 = map_to_rank(&acc_empty[0], 0), rel1 = map_to_rank(&acc_empty[1], 0);
         for (int u = pair; u < p.units && !*abort_flag; u += npairs) {
             int t, c0, c1, slot;
             hess_unit(p, nch, u, t, c0, c1, slot);
 #pragma unroll
-            for (int c = 0; c < 128; ++c) acc[c] = 0.f;
+            for (int c = 0; c < 128; ++c) HESS_ACC(c) = 0.f;
             bool first = true;
             int c = c0;
             for (; c < c1; ++c, ++ch) {
@@ -458,7 +472,7 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HessianParams p) {
                     float v[8];
                     tmem_ld8(ta + 8 * part8, v);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) acc[8 * part8 + i] += v[i];
+                    for (int i = 0; i < 8; ++i) HESS_ACC(8 * part8 + i) += v[i];
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -475,8 +489,8 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HessianParams p) {
                     float *Sr = hess_slot(p, slot) + (long long)rloc * p.n + 128 * h;
 #pragma unroll
                     for (int x = 0; x < 32; ++x) {
-                        float4 v = make_float4(2.f * acc[4 * x], 2.f * acc[4 * x + 1],
-                                               2.f * acc[4 * x + 2], 2.f * acc[4 * x + 3]);
+                        float4 v = make_float4(2.f * HESS_ACC(4 * x), 2.f * HESS_ACC(4 * x + 1),
+                                               2.f * HESS_ACC(4 * x + 2), 2.f * HESS_ACC(4 * x + 3));
                         if (first) *reinterpret_cast<float4 *>(Sr + 4 * x) = v;
                         else red_add_v4(Sr + 4 * x, v.x, v.y, v.z, v.w);
                     }
@@ -487,22 +501,23 @@ hessian_tc_kernel(const __grid_constant__ CUtensorMap xmap, HessianParams p) {
                         // the warp's whole 32 x 128 block is on or above the diagonal
 #pragma unroll
                         for (int x = 0; x < 32; ++x)
-                            red_add_v4(Hr + 4 * x, 2.f * acc[4 * x], 2.f * acc[4 * x + 1],
-                                       2.f * acc[4 * x + 2], 2.f * acc[4 * x + 3]);
+                            red_add_v4(Hr + 4 * x, 2.f * HESS_ACC(4 * x), 2.f * HESS_ACC(4 * x + 1),
+                                       2.f * HESS_ACC(4 * x + 2), 2.f * HESS_ACC(4 * x + 3));
                     } else if (col0 + 127 >= rbase) {
 #pragma unroll
                         for (int cc = 0; cc < 128; ++cc) {
                             const int col = col0 + cc;
-                            if (col >= row && col < p.n) red_add(Hr + cc, 2.f * acc[cc]);
+                            if (col >= row && col < p.n) red_add(Hr + cc, 2.f * HESS_ACC(cc));
                         }
                     }
                 }
                 first = false;
 #pragma unroll
-                for (int cc = 0; cc < 128; ++cc) acc[cc] = 0.f;
+                for (int cc = 0; cc < 128; ++cc) HESS_ACC(cc) = 0.f;
             }
             if (c < c1) break;  // left on an abort
         }
+#undef HESS_ACC
     }
     tc_fence_before();
     __syncthreads();

@@ -87,7 +87,9 @@ GPTQ_API uint64_t gptq_launch_count(void);
  * GPTQ (encyclopedia article), "Technical approach": the quantizer is driven by the
  * Hessian of the layer-wise squared error ||XW - XQ||^2, which is 2 X^T X.
  *   H       device, n x n fp32 row-major, caller-owned; accumulated into (zero it before
- *           the first chunk). On return both triangles hold the symmetric sum.
+ *           the first chunk). Only the upper triangle (diagonal included) is read; the
+ *           strictly lower one may serve as scratch during the call. On return both
+ *           triangles hold the symmetric sum.
  *   X       device, k x n row-major calibration chunk; x_dtype GPTQ_BF16 or GPTQ_F32.
  *           The base address must be 16-byte aligned; for GPTQ_BF16, n % 8 == 0.
  *   k, n    k >= 0 tokens (k == 0 is a no-op), 1 <= n <= 65536 features.

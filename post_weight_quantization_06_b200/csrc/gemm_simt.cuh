@@ -201,40 +201,58 @@ struct F64Epilogue {
 // C = alpha * op(A) op(B) (+ epilogue) accumulated in fp64 (64 x 64 tiles, 4 x 4 per thread).
 // For the products whose result is a small difference of large numbers or must keep the weak
 // directions of an ill-conditioned block: the orthonormalisation and Rayleigh-Ritz steps and
-// the Schur complement of the intrinsic-LoRA factor.
+// the Schur complement of the intrinsic-LoRA factor. The K loop stages 32-deep slabs through
+// shared memory with the next slab's global loads in flight. With gridDim.z > 1 the K range
+// is split: split z writes its fp64 partial sums to part[z] (M x N, dense) and
+// f64acc_reduce_kernel adds the splits in order and applies the epilogue.
+constexpr int F64_T = 64, F64_BK = 32;
+
 template <typename TA, typename TB, typename TC>
 __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, const TA *A,
                                                           long long lda, int ta, const TB *B,
                                                           long long ldb, int tb, TC *C,
                                                           long long ldc, double alpha,
-                                                          int b_upper, F64Epilogue ep) {
-    constexpr int T = 64, BK = 16;
+                                                          int b_upper, F64Epilogue ep,
+                                                          double *part, int kchunk) {
+    constexpr int T = F64_T, BK = F64_BK, PER = T * BK / 256;  // 8 elements per thread
     __shared__ double As[BK][T + 1];
     __shared__ double Bs[BK][T + 1];
     const int i0 = blockIdx.y * T, j0 = blockIdx.x * T;
     if (ep.c_upper && i0 >= j0 + T) return;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
     double acc[4][4] = {};
-    int kend = K;
+    int kbeg = blockIdx.z * kchunk, kend = min(K, kbeg + kchunk);
     if (b_upper) kend = min(kend, j0 + T);
-    for (int k0 = 0; k0 < kend; k0 += BK) {
-        for (int idx = tid; idx < T * BK; idx += 256) {
+    double ra[PER], rb[PER];
+    auto load = [&](int k0) {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int idx = tid + 256 * e;
             int r, kk;
             if (ta) { kk = idx / T; r = idx % T; } else { r = idx / BK; kk = idx % BK; }
             const int gi = i0 + r, gk = k0 + kk;
-            As[kk][r] = (gi < M && gk < kend)
-                            ? to_f64(ta ? A[(long long)gk * lda + gi] : A[(long long)gi * lda + gk])
-                            : 0.0;
+            ra[e] = (gi < M && gk < kend)
+                        ? to_f64(ta ? A[(long long)gk * lda + gi] : A[(long long)gi * lda + gk])
+                        : 0.0;
             int c;
             if (tb) { c = idx / BK; kk = idx % BK; } else { kk = idx / T; c = idx % T; }
-            const int gj = j0 + c;
-            const int gk2 = k0 + kk;
-            Bs[kk][c] = (gj < N && gk2 < kend && (!b_upper || gk2 <= gj))
-                            ? to_f64(tb ? B[(long long)gj * ldb + gk2] : B[(long long)gk2 * ldb + gj])
-                            : 0.0;
+            const int gj = j0 + c, gk2 = k0 + kk;
+            rb[e] = (gj < N && gk2 < kend && (!b_upper || gk2 <= gj))
+                        ? to_f64(tb ? B[(long long)gj * ldb + gk2] : B[(long long)gk2 * ldb + gj])
+                        : 0.0;
+        }
+    };
+    if (kbeg < kend) load(kbeg);
+    for (int k0 = kbeg; k0 < kend; k0 += BK) {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) {
+            const int idx = tid + 256 * e;
+            if (ta) As[idx / T][idx % T] = ra[e]; else As[idx % BK][idx / BK] = ra[e];
+            if (tb) Bs[idx % BK][idx / BK] = rb[e]; else Bs[idx / T][idx % T] = rb[e];
         }
         __syncthreads();
-#pragma unroll
+        if (k0 + BK < kend) load(k0 + BK);  // next slab in flight during the FMAs
+#pragma unroll 8
         for (int kk = 0; kk < BK; ++kk) {
             double a[4], b[4];
 #pragma unroll
@@ -245,6 +263,20 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
                 for (int v = 0; v < 4; ++v) acc[u][v] = fma(a[u], b[v], acc[u][v]);
         }
         __syncthreads();
+    }
+    if (part) {
+        double *P = part + (long long)blockIdx.z * M * N;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int gi = i0 + ty + 16 * u;
+            if (gi >= M) continue;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const int gj = j0 + tx + 16 * v;
+                if (gj < N) P[(long long)gi * N + gj] = acc[u][v];
+            }
+        }
+        return;
     }
     const double dg = ep.diag ? (double)*ep.diag : 0.0;
 #pragma unroll
@@ -263,15 +295,67 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
     }
 }
 
+// C = alpha * sum_z part[z] (+ epilogue): the splits added in order, so the result does not
+// depend on scheduling.
+template <typename TC>
+__global__ void f64acc_reduce_kernel(int M, int N, int splits, const double *part, TC *C,
+                                     long long ldc, double alpha, F64Epilogue ep) {
+    const long long total = (long long)M * N;
+    const double dg = ep.diag ? (double)*ep.diag : 0.0;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int gi = (int)(idx / N), gj = (int)(idx % N);
+        if (ep.c_upper && gj < gi) continue;
+        double acc = 0.0;
+        for (int z = 0; z < splits; ++z) acc += part[(long long)z * total + idx];
+        double val = alpha * acc;
+        if (ep.Cin) val += ep.beta * (double)ep.Cin[(long long)gi * ep.ldcin + gj];
+        if (gi == gj) val += dg;
+        C[(long long)gi * ldc + gj] = (TC)val;
+    }
+}
+
+// Scratch for split-K: `part` holds part_elems doubles (nullptr: no split).
+struct F64Split {
+    double *part = nullptr;
+    size_t part_elems = 0;
+};
+
 template <typename TA, typename TB, typename TC>
 inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, const TB *B,
                        long long ldb, int tb, TC *C, long long ldc, double alpha, cudaStream_t s,
-                       int b_upper = 0, F64Epilogue ep = F64Epilogue()) {
+                       int b_upper = 0, F64Epilogue ep = F64Epilogue(), F64Split sp = F64Split()) {
     if (M <= 0 || N <= 0) return GPTQ_OK;
-    dim3 grid(ceil_div(N, 64), ceil_div(M, 64));
+    dim3 grid(ceil_div(N, F64_T), ceil_div(M, F64_T), 1);
+    // split K when the output tiles fill less than two waves and K is long
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long tiles = (long long)grid.x * grid.y;
+    int splits = 1;
+    if (sp.part && tiles < 2LL * sms && K >= 2048) {
+        splits = (int)((2LL * sms + tiles - 1) / tiles);
+        if (splits > K / 512) splits = K / 512;
+        if (splits > 16) splits = 16;
+        while (splits > 1 && (size_t)splits * M * N > sp.part_elems) --splits;
+    }
+    int kchunk = K;
+    if (splits > 1) {
+        kchunk = ceil_div(ceil_div(K, splits), F64_BK) * F64_BK;
+        splits = ceil_div(K, kchunk);
+    }
+    grid.z = splits;
     gemm_f64acc_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, lda, ta, B, ldb, tb, C, ldc,
-                                                        alpha, b_upper, ep);
-    return launch_status();
+                                                        alpha, b_upper, ep,
+                                                        splits > 1 ? sp.part : nullptr, kchunk);
+    if (int st = launch_status()) return st;
+    if (splits > 1) {
+        const long long total = (long long)M * N;
+        const int blocks = (int)((total + 255) / 256 < 4LL * sms ? (total + 255) / 256 : 4LL * sms);
+        f64acc_reduce_kernel<TC><<<blocks, 256, 0, s>>>(M, N, splits, sp.part, C, ldc, alpha, ep);
+        return launch_status();
+    }
+    return GPTQ_OK;
 }
 
 // Copy the upper triangle of an n x n matrix onto its lower triangle (32x32 smem tiles).

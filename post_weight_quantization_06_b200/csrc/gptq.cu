@@ -78,6 +78,8 @@ inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
         w.il.Yr = c.take<float>((size_t)n * r);
         w.il.C = c.take<double>((size_t)r * r);
         w.il.Ci = c.take<double>((size_t)r * r);
+        w.il.part_elems = (size_t)4 * n * p;
+        w.il.part = c.take<double>(w.il.part_elems);
     } else {
         std::memset(&w.il, 0, sizeof(w.il));
     }

@@ -68,6 +68,7 @@ __global__ __launch_bounds__(512) void jacobi_eig_kernel(const double *Tin, int 
     int *pj = pi + p / 2;
     __shared__ double red[2];
     const int tid = threadIdx.x, nt = blockDim.x;
+    const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
     for (int idx = tid; idx < p * p; idx += nt) {
         const int i = idx / p, j = idx % p;
         T[i * LD + j] = 0.5 * (Tin[i * p + j] + Tin[j * p + i]);
@@ -108,25 +109,28 @@ __global__ __launch_bounds__(512) void jacobi_eig_kernel(const double *Tin, int 
                 cs[k] = c; sn[k] = sv;
             }
             __syncthreads();
-            for (int idx = tid; idx < half * p; idx += nt) {
-                const int k = idx / p, l = idx % p;
+            // rows i, j of every pair (warp per pair, lanes along the row), then the columns
+            for (int k = warp; k < half; k += nwarps) {
                 const int i = pi[k], j = pj[k];
                 const double c = cs[k], sv = sn[k];
-                const double ti = T[i * LD + l], tj = T[j * LD + l];
-                T[i * LD + l] = c * ti - sv * tj;
-                T[j * LD + l] = sv * ti + c * tj;
+                for (int l = lane; l < p; l += 32) {
+                    const double ti = T[i * LD + l], tj = T[j * LD + l];
+                    T[i * LD + l] = c * ti - sv * tj;
+                    T[j * LD + l] = sv * ti + c * tj;
+                }
             }
             __syncthreads();
-            for (int idx = tid; idx < half * p; idx += nt) {
-                const int k = idx / p, l = idx % p;
+            for (int k = warp; k < half; k += nwarps) {
                 const int i = pi[k], j = pj[k];
                 const double c = cs[k], sv = sn[k];
-                const double ti = T[l * LD + i], tj = T[l * LD + j];
-                T[l * LD + i] = c * ti - sv * tj;
-                T[l * LD + j] = sv * ti + c * tj;
-                const float qi = Q[l * LD + i], qj = Q[l * LD + j];
-                Q[l * LD + i] = (float)(c * qi - sv * qj);
-                Q[l * LD + j] = (float)(sv * qi + c * qj);
+                for (int l = lane; l < p; l += 32) {
+                    const double ti = T[l * LD + i], tj = T[l * LD + j];
+                    T[l * LD + i] = c * ti - sv * tj;
+                    T[l * LD + j] = sv * ti + c * tj;
+                    const float qi = Q[l * LD + i], qj = Q[l * LD + j];
+                    Q[l * LD + i] = (float)(c * qi - sv * qj);
+                    Q[l * LD + j] = (float)(sv * qi + c * qj);
+                }
             }
             __syncthreads();
         }
@@ -210,7 +214,11 @@ struct ILWork {
     double *B12, *Y1;          // n x r: H V and H V C^-1/2
     float *Yr;                 // n x r: H V C^-1
     double *C, *Ci;            // r x r extra block and inverse UL factor
+    double *part;              // split-K partial sums of the fp64-accumulating products
+    size_t part_elems;         // 4 n p
 };
+
+inline F64Split il_split(const ILWork &w) { return F64Split{w.part, w.part_elems}; }
 
 constexpr int IL_ITERS_F32 = 4;   // power steps with fp32 accumulation
 constexpr int IL_ITERS_F64 = 1;   // then with fp64 accumulation, before Rayleigh-Ritz
@@ -218,9 +226,11 @@ constexpr int IL_ITERS_F64 = 1;   // then with fp64 accumulation, before Rayleig
 // dst = src Ubar^-T where src^T src = Ubar Ubar^T (Gram, factor and product in fp64):
 // dst has orthonormal columns spanning src.
 inline int cholqr_f64(const float *src, float *dst, int n, int p, ILWork &w, cudaStream_t s) {
-    if (int st = gemm_f64acc<float, float, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, float, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
     if (int st = diag_ul_inv<double>(w.G, p, w.Gi, p, p, 0, s)) return st;
-    return gemm_f64acc<float, double, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.0, s);
+    return gemm_f64acc<float, double, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.0,
+            s, 0, F64Epilogue(), il_split(w));
 }
 
 // Top-r eigenvectors of H (n x n) into V (n x r).
@@ -234,21 +244,25 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
         if (it < IL_ITERS_F32) {
             if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
         } else {
-            if (int st = gemm_f64acc<float, float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.0, s)) return st;
+            if (int st = gemm_f64acc<float, float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.0,
+                    s, 0, F64Epilogue(), il_split(w))) return st;
         }
         if (int st = cholqr_f64(w.Z, w.Y, n, p, w, s)) return st;
         if (int st = cholqr_f64(w.Y, w.Z, n, p, w, s)) return st;
         std::swap(w.Y, w.Z);
     }
     // Rayleigh-Ritz in fp64: Tm = Y^T (H Y)
-    if (int st = gemm_f64acc<float, float, double>(n, p, n, H, ldh, 0, w.Y, p, 0, w.HY, p, 1.0, s)) return st;
-    if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, float, double>(n, p, n, H, ldh, 0, w.Y, p, 0, w.HY, p, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
+    if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
     const size_t smem = jacobi_smem(p);
     cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     jacobi_eig_kernel<<<1, 512, smem, s>>>(w.Tm, p, r, w.Qsel, w.ev);
     GPTQ_CHECK_LAUNCH();
     // V = Y Qsel
-    if (int st = gemm_f64acc<float, float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
     sign_fix_kernel<<<r, 256, 0, s>>>(V, n, r);
     return launch_status();
 }
@@ -263,19 +277,24 @@ inline int il_factor(const float *H, long long ldh, int n, int r, const float *V
                      ILWork &w, cudaStream_t s) {
     const long long ldu = n + r;
     // B12 = H V (n x r), C = V^T B12 (r x r)
-    if (int st = gemm_f64acc<float, float, double>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.0, s)) return st;
-    if (int st = gemm_f64acc<float, double, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0, s)) return st;
+    if (int st = gemm_f64acc<float, float, double>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
+    if (int st = gemm_f64acc<float, double, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
     il_lambda_kernel<<<1, 1024, 0, s>>>(H, ldh, n, w.C, r, lambda_rel, lam);
     GPTQ_CHECK_LAUNCH();
     // C = Ubar Ubar^T, Ci = Ubar^-1, C^-1 = Ci^T Ci
     if (int st = diag_ul_inv<double>(w.C, r, w.Ci, r, r, 0, s)) return st;
     // Y1 = B12 Ci^T, Yr = Y1 Ci = B12 C^-1
-    if (int st = gemm_f64acc<double, double, double>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.0, s)) return st;
-    if (int st = gemm_f64acc<double, double, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.0, s, 1)) return st;
+    if (int st = gemm_f64acc<double, double, double>(n, r, r, w.B12, r, 0, w.Ci, r, 1, w.Y1, r, 1.0,
+            s, 0, F64Epilogue(), il_split(w))) return st;
+    if (int st = gemm_f64acc<double, double, float>(n, r, r, w.Y1, r, 0, w.Ci, r, 0, w.Yr, r, 1.0,
+            s, 1, F64Epilogue(), il_split(w))) return st;
     // S = H + l I - Y1 Y1^T (upper triangle), fp64 accumulation, fp32 result
     F64Epilogue ep;
     ep.Cin = H; ep.ldcin = ldh; ep.beta = 1.0; ep.diag = lam; ep.c_upper = 1;
-    if (int st = gemm_f64acc<double, double, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.0, s, 0, ep)) return st;
+    if (int st = gemm_f64acc<double, double, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.0,
+            s, 0, ep, il_split(w))) return st;
     cudaMemsetAsync(Uaug, 0, sizeof(float) * (size_t)n * ldu, s);
     if (int st = factor_ul_inverse(Awork, n, Uaug, ldu, n, T, s)) return st;
     // U12 = -U11 Yr

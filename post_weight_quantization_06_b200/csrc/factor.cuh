@@ -426,7 +426,9 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
         if (k > 0) {
             auto p = gemm_args<float, float>(bk, r, bk, Xkk, ldu, 0, A + r, lda, 1, Lt, lda, 1.f, 0.f);
             p.a_upper = 1;
-            if ((st = gemm_f32(p, fs->chain))) break;
+            // the chain's products are small (K = 128, at most 47 output tiles of 128): the SIMT
+            // kernel's 64-tiles start sooner and spread wider than the tensor-core pipeline
+            if ((st = gemm_simt(p, fs->chain))) break;
         }
         cudaEventRecord(fs->panel, fs->chain);
         if (k > 0) {
@@ -434,7 +436,7 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
             cudaStreamWaitEvent(fs->chain, fs->bulk_done, 0);  // bulk update of block k+1
             auto p = gemm_args<float, float>(r, FACTOR_NB, bk, Lt, lda, 1, Lt + r1, lda, 0, A + r1,
                                              lda, -1.f, 1.f);
-            if ((st = gemm_f32(p, fs->chain))) break;
+            if ((st = gemm_simt(p, fs->chain))) break;
             if (r1 > 0) {
                 cudaStreamWaitEvent(fs->bulk, fs->panel, 0);
                 auto q = gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);

@@ -30,6 +30,10 @@ il_* (intrinsic LoRA)           r = 0 equals plain GPTQ bit for bit; literal
                                 codes and R equal Babai on the augmented lattice;
                                 residual-based error bound
 pack_codes                      hand-derived golden words (tests/golden/pack_*.txt)
+olrc / bidup / refine_loop      OLrC's X (L R) equals the truncated SVD of X E^T and
+(OLrC + Bid-Up refinement)      its loss the dropped singular values; every Bid-Up
+                                decision is the brute-force best code for its
+                                coordinate; the loss history never increases
 ==============================  ==================================================
 """
 from .gptq import (
@@ -55,8 +59,11 @@ from .il import (
 )
 from .babai import ql_decomposition, babai_nearest_plane
 from .pack import pack_codes, unpack_codes
+from .refine import olrc, bidup, dequant, refine as refine_loop
+from .refine import data_loss_rows as lowrank_loss_rows
 
 __all__ = [
+    "olrc", "bidup", "dequant", "refine_loop", "lowrank_loss_rows",
     "hessian", "damp", "inverse_cholesky_upper", "minmax_grid", "sweep", "sweep_blocked",
     "gptq_layer", "replay", "regularised_loss_rows", "data_loss_rows",
     "top_singular_directions", "augmented_gram", "il_hessian", "eig_qr_factor",

@@ -8,6 +8,7 @@
  *   gptq_prepare_hinv         lambda = lambda_rel * mean(diag H); U upper with (H + lambda I)^-1 = U^T U
  *   gptq_quantize_layer       column sweep of W onto per-group min-max grids with error feedback
  *   gptq_il_quantize_layer    the same pass on the augmented calibration [X, X V_r]; returns Q, L = V_r, R
+ *   gptq_il_refine            OLrC + Bid-Up refinement rounds on a quantized layer: new L, R, codes
  *
  * Conventions shared by every entry point
  *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);
@@ -61,7 +62,8 @@ typedef enum {
     GPTQ_OP_HESSIAN = 0,
     GPTQ_OP_PREPARE_HINV = 1,
     GPTQ_OP_QUANTIZE = 2,
-    GPTQ_OP_IL_QUANTIZE = 3
+    GPTQ_OP_IL_QUANTIZE = 3,
+    GPTQ_OP_IL_REFINE = 4
 } gptq_op;
 
 /* Bytes of device workspace the entry point `op` needs for these sizes (0 if none).
@@ -206,6 +208,38 @@ GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64
                            uint32_t *codes, float *scales, uint8_t *zeros, float *L, float *R,
                            float *lambda_out, double *loss_out, void *workspace,
                            size_t ws_bytes, gptq_stream_t stream);
+
+/*
+ * OLrC + Bid-Up refinement of a quantized layer (GPTQ-intrinsic LoRA summary, section 4):
+ * `iters` rounds, each first OLrC (the best rank-r L, R for the current codes) and then
+ * Bid-Up (one pass of coordinate-wise code updates on the fixed grid for that L, R); the
+ * reconstruction error sum_o ||X (w_o - qhat_o - (R^T L^T)_o)||^2 never increases.
+ *   OLrC:   E = W - Qhat; P = top-r eigenvectors of E H E^T (m x m, by decreasing
+ *           eigenvalue, each column's largest-magnitude entry positive); R = P^T, L = E^T P.
+ *   Bid-Up: columns j = 0 .. n-1 in order, all rows at once; the code of (o, j) becomes
+ *           clip(rint(c + (d_o H)_j / (H_jj s)), 0, 2^bits - 1) with d_o = w_o - qhat_o -
+ *           (R^T L^T)_o and s the row's scale for j's group (scales and zero-points fixed);
+ *           columns with H_jj <= 0 are left alone.
+ *   W          device, m x n row-major, w_dtype GPTQ_BF16 or GPTQ_F32 (the original weights).
+ *   H          device, n x n fp32 raw Hessian 2 X^T X (undamped).
+ *   r          0 <= r <= 128, r < m, r < n (r == 0: Bid-Up rounds only, L and R unused).
+ *   bits, group_size  the grid of the codes (as in gptq_quantize_layer).
+ *   iters      >= 1 rounds.
+ *   codes      device, m x (n * bits / 32) uint32, packed as gptq_quantize_layer writes
+ *              them: read, and overwritten with the refined codes.
+ *   scales, zeros  device, the grid the codes refer to (read only).
+ *   L, R       device, n x r and r x m fp32: written with the last round's OLrC result.
+ *   loss_hist  device, 2 * iters doubles: the reconstruction error (with X^T X = H / 2)
+ *              after each round's OLrC and after its Bid-Up, in order.
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_IL_REFINE, m, n, r, 0) bytes.
+ * Argument errors: GPTQ_ERR_ARG, GPTQ_ERR_WORKSPACE (nothing enqueued). Device errors
+ * (non-positive pivot in the eigenvector step's orthonormalisation) go to the status word.
+ */
+GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
+                            int r, int bits, int group_size, int iters, uint32_t *codes,
+                            const float *scales, const uint8_t *zeros, float *L, float *R,
+                            double *loss_hist, void *workspace, size_t ws_bytes,
+                            gptq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,10 +19,11 @@ GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, -1, -2, -3
 GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
+GPTQ_OP_IL_REFINE = 4
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-            "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer")
+            "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine")
 
 
 class GptqError(RuntimeError):
@@ -51,6 +52,8 @@ def _load() -> ctypes.CDLL:
         "gptq_il_quantize_layer": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int,
                                            c_f, c_int, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p,
                                            c_sz, c_p]),
+        "gptq_il_refine": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int, c_int,
+                                   c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -198,6 +201,23 @@ def gptq_il_quantize_layer(W: torch.Tensor, H: torch.Tensor, r: int, bits: int, 
                                        _ptr(zeros), _ptr(L), _ptr(R), _ptr(lambda_out),
                                        _ptr(loss_out), _ptr(ws), ws.numel(), _stream(stream)),
            "gptq_il_quantize_layer")
+
+
+def gptq_il_refine(W: torch.Tensor, H: torch.Tensor, r: int, bits: int, group_size: int,
+                   iters: int, codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                   L: torch.Tensor | None, R: torch.Tensor | None, loss_hist: torch.Tensor,
+                   ws: torch.Tensor, stream=None):
+    _dev(W, "W")
+    _dev(H, "H", torch.float32)
+    _dev(codes, "codes", torch.int32)
+    _dev(scales, "scales", torch.float32)
+    _dev(zeros, "zeros", torch.uint8)
+    _dev(loss_hist, "loss_hist", torch.float64)
+    m, n = W.shape
+    _check(_lib.gptq_il_refine(_ptr(W), _dtype_code(W), m, n, _ptr(H), r, bits, group_size, iters,
+                               _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(L), _ptr(R),
+                               _ptr(loss_hist), _ptr(ws), ws.numel(), _stream(stream)),
+           "gptq_il_refine")
 
 
 # ------------------------------------------------------------------------------------------

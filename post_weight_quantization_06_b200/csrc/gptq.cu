@@ -8,6 +8,7 @@
 #include "factor.cuh"
 #include "quant.cuh"
 #include "il.cuh"
+#include "refine.cuh"
 #include "hessian_tc.cuh"
 
 namespace gptq {
@@ -57,6 +58,44 @@ struct IlWs {
     float *Uaug, *lam_dummy;
     ILWork il;
 };
+// Work arrays of the top-r eigenvector step on a dim x dim matrix.
+inline ILWork carve_ilwork(Carver &c, long long dim, int r) {
+    ILWork w;
+    const int p = il_block_p((int)dim, r);
+    w.Y = c.take<float>((size_t)dim * p);
+    w.Z = c.take<float>((size_t)dim * p);
+    w.Qsel = c.take<float>((size_t)p * r);
+    w.HY = c.take<double>((size_t)dim * p);
+    w.Tm = c.take<double>((size_t)p * p);
+    w.ev = c.take<double>((size_t)p);
+    w.G = c.take<double>((size_t)p * p);
+    w.Gi = c.take<double>((size_t)p * p);
+    w.B12 = c.take<double>((size_t)dim * r);
+    w.Y1 = c.take<double>((size_t)dim * r);
+    w.Yr = c.take<float>((size_t)dim * r);
+    w.C = c.take<double>((size_t)r * r);
+    w.Ci = c.take<double>((size_t)r * r);
+    w.part_elems = (size_t)4 * dim * p;
+    w.part = c.take<double>(w.part_elems);
+    return w;
+}
+
+inline RefineWs carve_refine(Carver &c, long long m, long long n, int r) {
+    RefineWs w;
+    w.E = c.take<float>((size_t)m * n);
+    w.Gm = c.take<float>((size_t)m * n);
+    w.D = c.take<float>((size_t)m * n);
+    w.Bm = c.take<float>((size_t)m * m);
+    w.P = c.take<float>((size_t)m * (r > 0 ? r : 1));
+    w.Z = c.take<float>((size_t)(r > 0 ? r : 1) * n);
+    w.Err = c.take<float>((size_t)m * BIDUP_B);
+    w.c8 = c.take<uint8_t>((size_t)m * n);
+    w.rowloss = c.take<double>((size_t)m);
+    if (r > 0) w.il = carve_ilwork(c, m, r);
+    else std::memset(&w.il, 0, sizeof(w.il));
+    return w;
+}
+
 inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
     IlWs w;
     w.q = carve_quant(c, m, n + r, B);
@@ -64,22 +103,7 @@ inline IlWs carve_il(Carver &c, long long m, long long n, int r, int B) {
     w.Uaug = c.take<float>((size_t)n * (n + r));
     w.lam_dummy = c.take<float>(1);
     if (r > 0) {
-        const int p = il_block_p((int)n, r);
-        w.il.Y = c.take<float>((size_t)n * p);
-        w.il.Z = c.take<float>((size_t)n * p);
-        w.il.Qsel = c.take<float>((size_t)p * r);
-        w.il.HY = c.take<double>((size_t)n * p);
-        w.il.Tm = c.take<double>((size_t)p * p);
-        w.il.ev = c.take<double>((size_t)p);
-        w.il.G = c.take<double>((size_t)p * p);
-        w.il.Gi = c.take<double>((size_t)p * p);
-        w.il.B12 = c.take<double>((size_t)n * r);
-        w.il.Y1 = c.take<double>((size_t)n * r);
-        w.il.Yr = c.take<float>((size_t)n * r);
-        w.il.C = c.take<double>((size_t)r * r);
-        w.il.Ci = c.take<double>((size_t)r * r);
-        w.il.part_elems = (size_t)4 * n * p;
-        w.il.part = c.take<double>(w.il.part_elems);
+        w.il = carve_ilwork(c, n, r);
     } else {
         std::memset(&w.il, 0, sizeof(w.il));
     }
@@ -187,6 +211,10 @@ GPTQ_API size_t gptq_workspace_size(int op, int64_t m, int64_t n, int r, int blo
         case GPTQ_OP_IL_QUANTIZE:
             if (m < 1 || r < 0) return 0;
             carve_il(c, m, n, r, block_size > 0 ? block_size : 128);
+            return c.off;
+        case GPTQ_OP_IL_REFINE:
+            if (m < 1 || r < 0) return 0;
+            carve_refine(c, m, n, r);
             return c.off;
         default:
             return 0;
@@ -325,6 +353,39 @@ GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64
         return launch_status();
     }
     return GPTQ_OK;
+}
+
+GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
+                            int r, int bits, int group_size, int iters, uint32_t *codes,
+                            const float *scales, const uint8_t *zeros, float *L, float *R,
+                            double *loss_hist, void *workspace, size_t ws_bytes,
+                            gptq_stream_t stream) {
+    if (!W || !H || !codes || !scales || !zeros || !loss_hist) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (!valid_quant_args(m, n, bits, group_size, 128)) return GPTQ_ERR_ARG;
+    if (r < 0 || r > IL_MAX_R || r >= n || r >= m) return GPTQ_ERR_ARG;
+    if (r > 0 && (!L || !R)) return GPTQ_ERR_ARG;
+    if (iters < 1) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_IL_REFINE, m, n, r, 0);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(workspace);
+    RefineWs w = carve_refine(c, m, n, r);
+    const int gs = group_size > 0 ? group_size : (int)n;
+    const long long words = n * bits / 32;
+    const int blocks = (int)std::min<long long>((m * n + 255) / 256, 148LL * 8);
+    refine_unpack_kernel<<<blocks, 256, 0, s>>>(codes, words, (int)m, (int)n, bits, w.c8, n);
+    GPTQ_CHECK_LAUNCH();
+    int st;
+    if (w_dtype == GPTQ_BF16)
+        st = il_refine(static_cast<const __nv_bfloat16 *>(W), (int)m, (int)n, H, r, bits, gs,
+                       iters, scales, zeros, L, R, loss_hist, w, s);
+    else
+        st = il_refine(static_cast<const float *>(W), (int)m, (int)n, H, r, bits, gs, iters,
+                       scales, zeros, L, R, loss_hist, w, s);
+    if (st) return st;
+    refine_pack_kernel<<<blocks, 256, 0, s>>>(w.c8, n, (int)m, (int)n, bits, codes, words);
+    return launch_status();
 }
 
 }  // extern "C"

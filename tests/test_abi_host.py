@@ -20,7 +20,7 @@ def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-        "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer"])
+        "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -60,8 +60,11 @@ def test_workspace_sizes():
     il0 = g.gptq_workspace_size(g.GPTQ_OP_IL_QUANTIZE, 2048, 6144, 0, 128)
     il = g.gptq_workspace_size(g.GPTQ_OP_IL_QUANTIZE, 2048, 6144, 64, 128)
     assert il > il0 >= q + f
+    rf = g.gptq_workspace_size(g.GPTQ_OP_IL_REFINE, 2048, 6144, 64, 0)
+    assert rf >= 3 * 2048 * 6144 * 4 + 2048 * 2048 * 4
+    assert g.gptq_workspace_size(g.GPTQ_OP_IL_REFINE, 2048, 6144, 0, 0) < rf
     assert g.gptq_workspace_size(99, 1, 1) == 0
-    for v in (f, q, il0, il):
+    for v in (f, q, il0, il, rf):
         assert v % 256 == 0
 
 
@@ -124,6 +127,26 @@ def test_il_rejects_bad_arguments(r, L, lam):
     st = _lib().gptq_il_quantize_layer(P, 1, 64, 256, P, r, 4, 128, ctypes.c_float(lam), 128,
                                        P, P, P, L, P, P, NULL, ctypes.c_void_p(1 << 20), need, NULL)
     assert st == -1
+
+
+@pytest.mark.parametrize("m,r,iters,loss,bits", [(64, -1, 1, P, 4), (64, 129, 1, P, 4),
+                                                 (64, 64, 1, P, 4), (8, 16, 1, P, 4),
+                                                 (64, 4, 0, P, 4), (64, 4, 1, NULL, 4),
+                                                 (64, 4, 1, P, 1)])
+def test_refine_rejects_bad_arguments(m, r, iters, loss, bits):
+    import post_weight_quantization_06_b200 as g
+    need = g.gptq_workspace_size(g.GPTQ_OP_IL_REFINE, m, 256, max(r, 0), 0)
+    st = _lib().gptq_il_refine(P, 1, m, 256, P, r, bits, 128, iters, P, P, P, P, P, loss,
+                               ctypes.c_void_p(1 << 20), need, NULL)
+    assert st == -1
+
+
+def test_refine_rejects_a_small_workspace():
+    import post_weight_quantization_06_b200 as g
+    need = g.gptq_workspace_size(g.GPTQ_OP_IL_REFINE, 64, 256, 4, 0)
+    st = _lib().gptq_il_refine(P, 1, 64, 256, P, 4, 4, 128, 1, P, P, P, P, P, P,
+                               ctypes.c_void_p(1 << 20), need - 256, NULL)
+    assert st == -6
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):

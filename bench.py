@@ -48,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
+    ap.add_argument("--refine-rounds", type=int, default=2,
+                    help="OLrC + Bid-Up rounds timed after the pass (reported apart, 0: none)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="use only the first TOKENS calibration rows (small profiling cases)")
     return ap.parse_args(argv)
@@ -292,6 +294,38 @@ def run_e2e(g, layer, lp, steps, warmup, chunk_tokens=32768):
     return ms, h2d, d2h
 
 
+def run_refine(g, layer, lp, rounds):
+    """OLrC + Bid-Up refinement (gptq_il_refine) of the pass's output, timed apart from the
+    pass: `rounds` rounds on the codes the last timed step produced, with the same H."""
+    dev = layer.W.device
+    m, n, r = layer.m, layer.n, layer.r
+    ws = g.workspace(g.GPTQ_OP_IL_REFINE, m, n, r, 0, dev)
+    Lr = torch.empty(n, max(r, 1), device=dev)
+    Rr = torch.empty(max(r, 1), m, device=dev)
+    hist = torch.empty(2 * rounds, dtype=torch.float64, device=dev)
+    start = lp.codes.clone()
+    codes = start.clone()
+    s = lp.s
+
+    def once():
+        codes.copy_(start)
+        g.gptq_il_refine(layer.W, lp.H, r, layer.bits, layer.group_size, rounds, codes, lp.scales,
+                         lp.zeros, Lr if r else None, Rr if r else None, hist, ws, stream=s)
+
+    with torch.cuda.stream(s):
+        once()                                   # warm-up
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        once()
+        e1.record(s)
+    torch.cuda.synchronize(dev)
+    h = hist.cpu().tolist()
+    changed = int((codes != start).sum().item())   # packed words that differ
+    return {"rounds": rounds, "ms": e0.elapsed_time(e1), "ms_per_round": e0.elapsed_time(e1) / rounds,
+            "loss_after_first_olrc": h[0], "loss_final": h[-1],
+            "loss_drop": (h[0] - h[-1]) / h[0] if h[0] else 0.0, "code_words_changed": changed}
+
+
 def cpu_baseline(layer, budget_s: float):
     """The fp64 oracle as it stands, on a bounded sample of the same layer, on the host cores:
     Hessian over a slice of the tokens, the full n x n factor, the sweep over a few rows;
@@ -398,6 +432,8 @@ def bench_ours(args):
         peak, peak_src = 1400.0, "fallback (bf16 sustained)"
     h_tflops = hessian_flops(layer) / (stage[0] * 1e-3) / 1e12
 
+    refine = run_refine(g, layer, lp, args.refine_rounds) if args.refine_rounds > 0 else None
+
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = run_e2e(g, layer, lp, max(1, args.steps), 2)
@@ -435,6 +471,8 @@ def bench_ours(args):
         }
         if e2e:
             out["e2e"] = e2e
+        if refine:
+            out["refine"] = refine
         if not args.no_cpu_baseline and world == 1:
             out["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
         print(json.dumps(out))

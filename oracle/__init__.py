@@ -34,6 +34,9 @@ olrc / bidup / refine_loop      OLrC's X (L R) equals the truncated SVD of X E^T
 (OLrC + Bid-Up refinement)      its loss the dropped singular values; every Bid-Up
                                 decision is the brute-force best code for its
                                 coordinate; the loss history never increases
+rtn_quantize / quantize_lowrank every code is the brute-force nearest grid point;
+(4-bit L, 8-bit R)              re-quantizing the dequantized values is idempotent;
+                                grid and packing pinned as above
 ==============================  ==================================================
 """
 from .gptq import (
@@ -61,9 +64,11 @@ from .babai import ql_decomposition, babai_nearest_plane
 from .pack import pack_codes, unpack_codes
 from .refine import olrc, bidup, dequant, refine as refine_loop
 from .refine import data_loss_rows as lowrank_loss_rows
+from .lowbit import rtn_quantize, quantize_lowrank
 
 __all__ = [
-    "olrc", "bidup", "dequant", "refine_loop", "lowrank_loss_rows",
+    "olrc", "bidup", "dequant", "refine_loop", "lowrank_loss_rows", "rtn_quantize",
+    "quantize_lowrank",
     "hessian", "damp", "inverse_cholesky_upper", "minmax_grid", "sweep", "sweep_blocked",
     "gptq_layer", "replay", "regularised_loss_rows", "data_loss_rows",
     "top_singular_directions", "augmented_gram", "il_hessian", "eig_qr_factor",

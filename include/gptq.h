@@ -9,6 +9,7 @@
  *   gptq_quantize_layer       column sweep of W onto per-group min-max grids with error feedback
  *   gptq_il_quantize_layer    the same pass on the augmented calibration [X, X V_r]; returns Q, L = V_r, R
  *   gptq_il_refine            OLrC + Bid-Up refinement rounds on a quantized layer: new L, R, codes
+ *   gptq_quantize_lowrank     L and R stored at low precision (4-bit L, 8-bit R) on min-max grids
  *
  * Conventions shared by every entry point
  *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);
@@ -240,6 +241,28 @@ GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, co
                             const float *scales, const uint8_t *zeros, float *L, float *R,
                             double *loss_hist, void *workspace, size_t ws_bytes,
                             gptq_stream_t stream);
+
+/*
+ * Low-precision storage of the low-rank factors (GPTQ-intrinsic LoRA summary, "Main
+ * results": quantizing L to 4 bits and R to 8 bits is often lossless). Round-to-nearest,
+ * no error feedback, onto the same per-group min-max grid the pass uses, each factor stored
+ * one neuron per row like the layer's weights:
+ *   L^T: r rows of n inputs, groups of group_size_L (0: one group per row), bits_L;
+ *   R^T: m rows of r inputs, one group per row, bits_R.
+ *   L, R        device, n x r and r x m fp32 (as gptq_il_quantize_layer / gptq_il_refine
+ *               write them), read only.
+ *   codes_L     device, r x (n * bits_L / 32) uint32; scales_L r x (n / group size) fp32;
+ *               zeros_L the same shape, uint8.
+ *   codes_R     device, m x (r * bits_R / 32) uint32; scales_R, zeros_R m x 1.
+ *   Codes are packed as gptq_quantize_layer packs them; the dequantized value of code c is
+ *   s (c - z). Requires 2 <= bits <= 8, n * bits_L and r * bits_R multiples of 32,
+ *   1 <= r <= 128.
+ * Argument errors: GPTQ_ERR_ARG (nothing enqueued).
+ */
+GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, int64_t m, int r,
+                                   int bits_L, int group_size_L, int bits_R, uint32_t *codes_L,
+                                   float *scales_L, uint8_t *zeros_L, uint32_t *codes_R,
+                                   float *scales_R, uint8_t *zeros_R, gptq_stream_t stream);
 
 #ifdef __cplusplus
 }

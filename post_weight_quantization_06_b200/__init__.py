@@ -23,7 +23,8 @@ GPTQ_OP_IL_REFINE = 4
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-            "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine")
+            "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
+            "gptq_quantize_lowrank")
 
 
 class GptqError(RuntimeError):
@@ -54,6 +55,8 @@ def _load() -> ctypes.CDLL:
                                            c_sz, c_p]),
         "gptq_il_refine": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_int, c_int, c_int,
                                    c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "gptq_quantize_lowrank": (c_int, [c_p, c_p, c_i64, c_i64, c_int, c_int, c_int, c_int,
+                                          c_p, c_p, c_p, c_p, c_p, c_p, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -218,6 +221,24 @@ def gptq_il_refine(W: torch.Tensor, H: torch.Tensor, r: int, bits: int, group_si
                                _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(L), _ptr(R),
                                _ptr(loss_hist), _ptr(ws), ws.numel(), _stream(stream)),
            "gptq_il_refine")
+
+
+def gptq_quantize_lowrank(L: torch.Tensor, R: torch.Tensor, bits_L: int, group_size_L: int,
+                          bits_R: int, codes_L: torch.Tensor, scales_L: torch.Tensor,
+                          zeros_L: torch.Tensor, codes_R: torch.Tensor, scales_R: torch.Tensor,
+                          zeros_R: torch.Tensor, stream=None):
+    _dev(L, "L", torch.float32)
+    _dev(R, "R", torch.float32)
+    for t, name, dt in ((codes_L, "codes_L", torch.int32), (scales_L, "scales_L", torch.float32),
+                        (zeros_L, "zeros_L", torch.uint8), (codes_R, "codes_R", torch.int32),
+                        (scales_R, "scales_R", torch.float32), (zeros_R, "zeros_R", torch.uint8)):
+        _dev(t, name, dt)
+    n, r = L.shape
+    m = R.shape[1]
+    _check(_lib.gptq_quantize_lowrank(_ptr(L), _ptr(R), n, m, r, bits_L, group_size_L, bits_R,
+                                      _ptr(codes_L), _ptr(scales_L), _ptr(zeros_L), _ptr(codes_R),
+                                      _ptr(scales_R), _ptr(zeros_R), _stream(stream)),
+           "gptq_quantize_lowrank")
 
 
 # ------------------------------------------------------------------------------------------

@@ -388,4 +388,26 @@ GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, co
     return launch_status();
 }
 
+GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, int64_t m, int r,
+                                   int bits_L, int group_size_L, int bits_R, uint32_t *codes_L,
+                                   float *scales_L, uint8_t *zeros_L, uint32_t *codes_R,
+                                   float *scales_R, uint8_t *zeros_R, gptq_stream_t stream) {
+    if (!L || !R || !codes_L || !scales_L || !zeros_L || !codes_R || !scales_R || !zeros_R)
+        return GPTQ_ERR_ARG;
+    if (n < 1 || m < 1 || r < 1 || r > IL_MAX_R || n > 65536 || m > (1LL << 30)) return GPTQ_ERR_ARG;
+    if (bits_L < 2 || bits_L > 8 || bits_R < 2 || bits_R > 8) return GPTQ_ERR_ARG;
+    if ((n * bits_L) % 32 || ((long long)r * bits_R) % 32) return GPTQ_ERR_ARG;
+    if (group_size_L < 0 || (group_size_L > 0 && n % group_size_L)) return GPTQ_ERR_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int gsL = group_size_L > 0 ? group_size_L : (int)n;
+    // L^T: r rows of n inputs; R^T: m rows of r inputs (one group)
+    rtn_rows_kernel<<<ceil_div(r, 8), 256, 0, s>>>(L, 1, r, r, (int)n, bits_L, gsL, codes_L,
+                                                   n * bits_L / 32, scales_L, zeros_L,
+                                                   (int)(n / gsL));
+    GPTQ_CHECK_LAUNCH();
+    rtn_rows_kernel<<<ceil_div(m, 8), 256, 0, s>>>(R, 1, m, (int)m, r, bits_R, r, codes_R,
+                                                   (long long)r * bits_R / 32, scales_R, zeros_R, 1);
+    return launch_status();
+}
+
 }  // extern "C"

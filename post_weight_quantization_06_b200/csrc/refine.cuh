@@ -313,4 +313,54 @@ inline int il_refine(const TW *W, int m, int n, const float *H, int r, int bits,
     return GPTQ_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// Low-precision storage of the low-rank factors (GPTQ-intrinsic LoRA summary, "Main
+// results": 4-bit L and 8-bit R are often lossless): round-to-nearest onto the pass's
+// per-group min-max grid, each factor stored one neuron per row. A(row, col) =
+// A[row * rs + col * cs] (L^T: rs = 1, cs = r; R^T: rs = 1, cs = m). One warp per row:
+// group ranges by warp reduction, the grid by the sweep's own rule (grid_from_range), then
+// the packed words, each lane recomputing the codes of the words it writes.
+// ---------------------------------------------------------------------------------------
+__global__ void rtn_rows_kernel(const float *A, long long rs, long long cs, int rows, int cols,
+                                int bits, int gs, uint32_t *codes, long long ldw, float *scales,
+                                uint8_t *zeros, int G) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    if (warp >= rows) return;
+    const float fmaxq = (float)((1 << bits) - 1);
+    const float *a = A + (long long)warp * rs;
+    for (int g = 0; g < G; ++g) {
+        float mn = INFINITY, mx = -INFINITY;
+        for (int c = g * gs + lane; c < min(cols, (g + 1) * gs); c += 32) {
+            const float x = a[(long long)c * cs];
+            mn = fminf(mn, x);
+            mx = fmaxf(mx, x);
+        }
+        mn = warp_min(mn);
+        mx = warp_max(mx);
+        float s, is, z;
+        grid_from_range(mn, mx, fmaxq, s, is, z);
+        if (lane == 0) {
+            scales[(long long)warp * G + g] = s;
+            zeros[(long long)warp * G + g] = (uint8_t)z;
+        }
+    }
+    __syncwarp();
+    const int words = cols * bits / 32;
+    for (int w = lane; w < words; w += 32) {
+        const int bit0 = 32 * w;
+        const int cfirst = bit0 / bits, clast = min(cols - 1, (bit0 + 31) / bits);
+        uint32_t word = 0;
+        for (int c = cfirst; c <= clast; ++c) {
+            const int g = c / gs;
+            const float s = scales[(long long)warp * G + g];
+            const float z = (float)zeros[(long long)warp * G + g];
+            const float v = fmaf(a[(long long)c * cs], __frcp_rn(s), z);
+            const uint32_t code = (uint32_t)fminf(fmaxf(rintf(v), 0.f), fmaxq);
+            const int pos = c * bits - bit0;
+            word |= pos >= 0 ? (code << pos) : (code >> (-pos));
+        }
+        codes[(long long)warp * ldw + w] = word;
+    }
+}
+
 }  // namespace gptq

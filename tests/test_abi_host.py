@@ -20,7 +20,8 @@ def test_header_declares_the_boundary():
     assert _declared() == sorted([
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
-        "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine"])
+        "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
+        "gptq_quantize_lowrank"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -147,6 +148,15 @@ def test_refine_rejects_a_small_workspace():
     st = _lib().gptq_il_refine(P, 1, 64, 256, P, 4, 4, 128, 1, P, P, P, P, P, P,
                                ctypes.c_void_p(1 << 20), need - 256, NULL)
     assert st == -6
+
+
+@pytest.mark.parametrize("n,r,bL,gL,bR", [(256, 0, 4, 128, 8), (256, 129, 4, 128, 8),
+                                           (256, 64, 1, 128, 8), (256, 64, 4, 100, 8),
+                                           (12, 64, 4, 0, 8), (256, 3, 4, 128, 8),
+                                           (256, 64, 4, 128, 9)])
+def test_lowrank_quantize_rejects_bad_arguments(n, r, bL, gL, bR):
+    st = _lib().gptq_quantize_lowrank(P, P, n, 64, r, bL, gL, bR, P, P, P, P, P, P, NULL)
+    assert st == -1
 
 
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):

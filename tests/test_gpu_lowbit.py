@@ -1,0 +1,65 @@
+"""Low-precision storage of L (4-bit) and R (8-bit) on the GPU against the fp64 oracle
+(GPTQ-intrinsic LoRA summary, "Main results"). Inputs are the device IL pass's own L, R."""
+import numpy as np
+import pytest
+import torch
+
+import datagen
+import oracle
+from gpu_parity import CODE_AGREE, CODE_BAND, np64, unpack
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def g():
+    import post_weight_quantization_06_b200 as lib
+    return lib
+
+
+def _judge(label, q, codes_gpu, scales_gpu, zeros_gpu):
+    v = q["v"]
+    mism = codes_gpu != q["codes"]
+    agree = 1.0 - mism.sum() / mism.size
+    worst = float(np.abs(np.abs(v[mism] - codes_gpu[mism]) - 0.5).max()) if mism.any() else 0.0
+    srel = np.abs(scales_gpu - q["scales"]).max() / np.abs(q["scales"]).max()
+    print(f"{label}: codes agree {agree:.6f} ({int(mism.sum())} differ, worst distance "
+          f"{worst:.2e} steps); scales max rel err {srel:.2e}; zeros differ "
+          f"{int((zeros_gpu != q['zeros']).sum())}")
+    assert agree >= CODE_AGREE and worst < CODE_BAND and srel <= 1e-6
+
+
+@pytest.mark.parametrize("r,gsL", [(16, 128), (16, 0), (32, 64)])
+def test_lowrank_factors_at_4_and_8_bits(g, r, gsL):
+    L = datagen.lowrank(device=DEV, scale=0.0625, r=16)
+    n, m = L.n, L.m
+    H = torch.zeros(n, n, device=DEV)
+    g.gptq_hessian_accumulate(H, L.X)
+    out = g.quantize_layer(L.W, H=H, bits=L.bits, group_size=L.group_size,
+                           lambda_rel=L.lambda_rel, r=r, intrinsic=True)
+    Lg, Rg = out["L"], out["R"]
+    GL = n // gsL if gsL else 1
+    cL = torch.empty(r, n * 4 // 32, dtype=torch.int32, device=DEV)
+    sL = torch.empty(r, GL, device=DEV)
+    zL = torch.empty(r, GL, dtype=torch.uint8, device=DEV)
+    cR = torch.empty(m, r * 8 // 32, dtype=torch.int32, device=DEV)
+    sR = torch.empty(m, 1, device=DEV)
+    zR = torch.empty(m, 1, dtype=torch.uint8, device=DEV)
+    g.gptq_quantize_lowrank(Lg, Rg, 4, gsL, 8, cL, sL, zL, cR, sR, zR)
+    g.gptq_sync_status()
+    Ld, Rd = np64(Lg), np64(Rg)
+    q = oracle.quantize_lowrank(Ld, Rd, bits_L=4, group_size_L=gsL, bits_R=8)
+    _judge(f"L^T r={r} g{gsL} 4-bit", q["L"], unpack(cL, 4, n), np64(sL), zL.cpu().numpy())
+    _judge(f"R^T r={r} 8-bit", q["R"], unpack(cR, 8, r), np64(sR), zR.cpu().numpy())
+    # reconstruction error of the layer with the stored factors, against fp32 factors
+    G = np64(H) / 2
+    Qhat = oracle.dequant(unpack(out["codes"], L.bits, n), np64(out["scales"]),
+                          out["zeros"].cpu().numpy(), L.group_size)
+    W = np64(L.W)
+    full = oracle.lowrank_loss_rows(W, Qhat, Ld, Rd, G).sum()
+    low = oracle.lowrank_loss_rows(W, Qhat, q["L_hat"], q["R_hat"], G).sum()
+    none = oracle.lowrank_loss_rows(W, Qhat, None, None, G).sum()
+    print(f"r={r} g{gsL}: reconstruction error with fp32 L, R {full:.6e}; 4-bit L / 8-bit R "
+          f"{low:.6e} ({low / full - 1:+.2%}); without the low-rank term {none:.6e}")
+    assert low < none

@@ -37,6 +37,9 @@ olrc / bidup / refine_loop      OLrC's X (L R) equals the truncated SVD of X E^T
 rtn_quantize / quantize_lowrank every code is the brute-force nearest grid point;
 (4-bit L, 8-bit R)              re-quantizing the dequantized values is idempotent;
                                 grid and packing pinned as above
+gptq2d_* (two-sided rounding)   anti-diagonal sweep equals the vectorised sweep and
+                                Babai nearest plane on the basis B^T (x) A; with
+                                B = I it is the one-sided sweep of every column
 ==============================  ==================================================
 """
 from .gptq import (
@@ -65,10 +68,12 @@ from .pack import pack_codes, unpack_codes
 from .refine import olrc, bidup, dequant, refine as refine_loop
 from .refine import data_loss_rows as lowrank_loss_rows
 from .lowbit import rtn_quantize, quantize_lowrank
+from .gptq2d import adaptive_round_1d, gptq2d_vectorized, gptq2d_antidiagonal, two_sided_loss
 
 __all__ = [
     "olrc", "bidup", "dequant", "refine_loop", "lowrank_loss_rows", "rtn_quantize",
-    "quantize_lowrank",
+    "quantize_lowrank", "adaptive_round_1d", "gptq2d_vectorized", "gptq2d_antidiagonal",
+    "two_sided_loss",
     "hessian", "damp", "inverse_cholesky_upper", "minmax_grid", "sweep", "sweep_blocked",
     "gptq_layer", "replay", "regularised_loss_rows", "data_loss_rows",
     "top_singular_directions", "augmented_gram", "il_hessian", "eig_qr_factor",

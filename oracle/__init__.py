@@ -40,6 +40,9 @@ rtn_quantize / quantize_lowrank every code is the brute-force nearest grid point
 gptq2d_* (two-sided rounding)   anti-diagonal sweep equals the vectorised sweep and
                                 Babai nearest plane on the basis B^T (x) A; with
                                 B = I it is the one-sided sweep of every column
+gptq2d_residuals                closed form X - Z = U_G^T E U_H: equals the sweep's
+                                recorded v - z; every |c| <= 1/2 for the sweep's Z
+                                and a Z moved by one step breaks it
 ==============================  ==================================================
 """
 from .gptq import (
@@ -68,12 +71,13 @@ from .pack import pack_codes, unpack_codes
 from .refine import olrc, bidup, dequant, refine as refine_loop
 from .refine import data_loss_rows as lowrank_loss_rows
 from .lowbit import rtn_quantize, quantize_lowrank
-from .gptq2d import adaptive_round_1d, gptq2d_vectorized, gptq2d_antidiagonal, two_sided_loss
+from .gptq2d import (adaptive_round_1d, gptq2d_antidiagonal, gptq2d_residuals, gptq2d_vectorized,
+                     reverse_cholesky_upper, two_sided_loss)
 
 __all__ = [
     "olrc", "bidup", "dequant", "refine_loop", "lowrank_loss_rows", "rtn_quantize",
     "quantize_lowrank", "adaptive_round_1d", "gptq2d_vectorized", "gptq2d_antidiagonal",
-    "two_sided_loss",
+    "two_sided_loss", "gptq2d_residuals", "reverse_cholesky_upper",
     "hessian", "damp", "inverse_cholesky_upper", "minmax_grid", "sweep", "sweep_blocked",
     "gptq_layer", "replay", "regularised_loss_rows", "data_loss_rows",
     "top_singular_directions", "augmented_gram", "il_hessian", "eig_qr_factor",

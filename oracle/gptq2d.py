@@ -47,14 +47,15 @@ def gptq2d_vectorized(X, G, H) -> np.ndarray:
     return adaptive_round_1d(X.reshape(-1, order="F"), UK).reshape(m, n, order="F")
 
 
-def gptq2d_antidiagonal(X, G, H) -> dict:
+def gptq2d_antidiagonal(X, G, H, force_Z=None) -> dict:
     """GPTQ-2D: stages s = 0 .. m+n-2 over the anti-diagonals, with two buffers:
       C[p, j] = sum_{i <= p} U_G[i, p] e_ij   (errors pushed down their column), and
       V[p, q] = sum_{j < q} C[p, j] U_H[j, q] (finished column buffers pushed along the row).
     Entry (p, q) is rounded from v = x_pq - V[p, q] - C[p, q] U_H[q, q], with C[p, q] then
     holding the errors of the entries above it in its column only. Its error
     e = (v - z) / (U_G[p, p] U_H[q, q]) is pushed down column q, after which C[p, q] is final
-    and is pushed along row p."""
+    and is pushed along row p. ``force_Z`` replaces the decisions (replay of another
+    implementation's trajectory); the pre-rounding values v are returned either way."""
     X = np.asarray(X, dtype=np.float64)
     m, n = X.shape
     UG, UH = inverse_cholesky_upper(G), inverse_cholesky_upper(H)
@@ -62,16 +63,40 @@ def gptq2d_antidiagonal(X, G, H) -> dict:
     V = np.zeros((m, n))
     Z = np.zeros((m, n), dtype=np.int64)
     E = np.zeros((m, n))
+    Vpre = np.zeros((m, n))
     for s in range(m + n - 1):
         for p in range(max(0, s - n + 1), min(m - 1, s) + 1):
             q = s - p
             v = X[p, q] - V[p, q] - C[p, q] * UH[q, q]
-            z = np.rint(v)
+            z = np.rint(v) if force_Z is None else float(force_Z[p, q])
             e = (v - z) / (UG[p, p] * UH[q, q])
-            Z[p, q], E[p, q] = int(z), e
+            Z[p, q], E[p, q], Vpre[p, q] = int(z), e, v
             C[p:, q] += UG[p, p:] * e
             V[p, q + 1:] += C[p, q] * UH[q, q + 1:]
-    return dict(Z=Z, E=E, UG=UG, UH=UH)
+    return dict(Z=Z, E=E, UG=UG, UH=UH, v=Vpre)
+
+
+def reverse_cholesky_upper(M) -> np.ndarray:
+    """Upper-triangular R with positive diagonal and M = R R^T: the Cholesky factor of M with
+    the index order reversed. R is the inverse of the upper factor U of M^-1 (M^-1 = U^T U)."""
+    M = np.asarray(M, dtype=np.float64)
+    L = np.linalg.cholesky(M[::-1, ::-1])
+    return np.ascontiguousarray(L[::-1, ::-1])
+
+
+def gptq2d_residuals(X, Z, G, H) -> np.ndarray:
+    """The scaled residual c = v - z of every decision, in closed form from Z alone.
+
+    Section 2: entry (p, q) receives U_G[i, p] U_H[j, q] e_ij from every earlier entry, so
+    X - Z = U_G^T E U_H (the entry's own error included). Hence E = Rg^T (X - Z) Rh with
+    Rg = U_G^-1, Rh = U_H^-1 (G = Rg Rg^T, H = Rh Rh^T), and c = e U_G[p,p] U_H[q,q] =
+    E[p, q] / (Rg[p,p] Rh[q,q]). The sweep's Z is the Babai point of the Kronecker basis:
+    every |c| <= 1/2 (the residual lies in the Gram-Schmidt parallelepiped), and no other
+    integer matrix has that property, so this checks a Z of any size."""
+    D = np.asarray(X, dtype=np.float64) - np.asarray(Z, dtype=np.float64)
+    Rg, Rh = reverse_cholesky_upper(G), reverse_cholesky_upper(H)
+    E = Rg.T @ D @ Rh
+    return E / np.outer(np.diag(Rg), np.diag(Rh))
 
 
 def two_sided_loss(X, Z, A, B) -> float:

@@ -84,3 +84,33 @@ def test_planted_mistakes_are_caught():
             V[p, q + 1:] += C[p, q] * UH[q, q + 1:]      # planted: row push before own error
             C[p:, q] += UG[p, p:] * e
     assert not np.array_equal(Z, good)
+
+
+@pytest.mark.parametrize("k,seed", [(1, 20), (6, 21), (40, 22)])
+def test_reverse_cholesky_factor(k, seed):
+    """R upper with M = R R^T, and R is the inverse of the upper factor of M^-1."""
+    g = np.random.default_rng(seed)
+    A = g.standard_normal((k, k)) + 2 * np.eye(k)
+    M = A @ A.T
+    R = oracle.reverse_cholesky_upper(M)
+    assert np.allclose(np.tril(R, -1), 0) and np.all(np.diag(R) > 0)
+    assert np.allclose(R @ R.T, M, rtol=1e-12, atol=1e-12 * np.abs(M).max())
+    U = oracle.inverse_cholesky_upper(M)
+    assert np.allclose(R @ U, np.eye(k), atol=1e-9)
+
+
+@pytest.mark.parametrize("m,n,seed", [(7, 11, 23), (12, 5, 24), (1, 9, 25)])
+def test_closed_form_residuals_match_the_sweep(m, n, seed):
+    """X - Z = U_G^T E U_H: the residuals computed from Z alone equal the sweep's own v - z,
+    lie in [-1/2, 1/2], and moving any single entry of Z by one step leaves that box."""
+    X, A, B, G, H = _problem(seed, m, n)
+    out = oracle.gptq2d_antidiagonal(X, G, H)
+    c = oracle.gptq2d_residuals(X, out["Z"], G, H)
+    assert np.allclose(c, out["v"] - out["Z"], atol=1e-9)
+    assert np.abs(c).max() <= 0.5 + 1e-12
+    g = np.random.default_rng(seed)
+    for _ in range(5):
+        Z2 = out["Z"].copy()
+        p, q = g.integers(m), g.integers(n)
+        Z2[p, q] += g.choice([-1, 1])
+        assert np.abs(oracle.gptq2d_residuals(X, Z2, G, H)).max() > 0.5

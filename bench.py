@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--refine-rounds", type=int, default=2,
                     help="OLrC + Bid-Up rounds timed after the pass (reported apart, 0: none)")
+    ap.add_argument("--no-gptq2d", action="store_true",
+                    help="skip the two-sided rounding (GPTQ-2D) timing reported under 'gptq2d'")
     ap.add_argument("--tokens", type=int, default=0,
                     help="use only the first TOKENS calibration rows (small profiling cases)")
     return ap.parse_args(argv)
@@ -326,6 +328,59 @@ def run_refine(g, layer, lp, rounds):
             "loss_drop": (h[0] - h[-1]) / h[0] if h[0] else 0.0, "code_words_changed": changed}
 
 
+SIMT_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max SM clock
+
+
+def run_gptq2d(g, dev, steps):
+    """Two-sided rounding (gptq_2d_round) of X 2048 x 6144 under G 2048^2, H 6144^2: the whole
+    call (both factorizations and the wavefront), and the factorizations alone through
+    gptq_prepare_hinv, so the wavefront's share is the difference."""
+    import datagen
+    P = datagen.two_sided(device=dev)
+    m, n = P.X.shape
+    Z = torch.empty(m, n, dtype=torch.int32, device=dev)
+    ws = g.workspace(g.GPTQ_OP_2D_ROUND, m, n, 0, 0, dev)
+    s = torch.cuda.Stream(device=dev)
+    UG, UH = torch.empty(m, m, device=dev), torch.empty(n, n, device=dev)
+    lam = torch.empty(1, device=dev)
+    wsf = g.workspace(g.GPTQ_OP_PREPARE_HINV, 0, max(m, n), 0, 0, dev)
+
+    def full():
+        g.gptq_2d_round(P.X, P.G, P.H, Z, None, ws, stream=s)
+
+    def factors():
+        g.gptq_prepare_hinv(P.G, 0.0, UG, lam, wsf, stream=s)
+        g.gptq_prepare_hinv(P.H, 0.0, UH, lam, wsf, stream=s)
+
+    def timed(fn, reps):
+        with torch.cuda.stream(s):
+            fn()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(reps):
+                fn()
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    reps = max(1, steps)
+    l0 = g.gptq_launch_count()
+    ms = timed(full, reps)
+    launches = (g.gptq_launch_count() - l0) // (reps + 1)
+    f_ms = timed(factors, reps)
+    st, _ = g.gptq_sync_status(s, raise_on_error=False)
+    wave_ms = ms - f_ms
+    flops = 2.0 * m * n * (m + n)         # every entry receives m + n feedback terms (one FMA each)
+    achieved = flops / (wave_ms * 1e-3) / 1e12
+    return {"workload": P.name + " fp32, G and H spectral Gram matrices", "ms": ms,
+            "entries_per_s": m * n / (ms * 1e-3), "factor_ms": f_ms, "wavefront_ms": wave_ms,
+            "launches_per_call": int(launches), "device_status": int(st),
+            "roofline": {"bound": "alu", "kernel": "wavefront (tile sweeps + band flushes), fp32 FMA",
+                         "achieved": achieved, "peak": SIMT_FP32_TFLOPS, "unit": "TFLOP/s",
+                         "frac": achieved / SIMT_FP32_TFLOPS,
+                         "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
+
+
 def cpu_baseline(layer, budget_s: float):
     """The fp64 oracle as it stands, on a bounded sample of the same layer, on the host cores:
     Hessian over a slice of the tokens, the full n x n factor, the sweep over a few rows;
@@ -434,6 +489,8 @@ def bench_ours(args):
 
     refine = run_refine(g, layer, lp, args.refine_rounds) if args.refine_rounds > 0 else None
 
+    two_d = run_gptq2d(g, dev, args.steps) if not args.no_gptq2d else None
+
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = run_e2e(g, layer, lp, max(1, args.steps), 2)
@@ -473,6 +530,8 @@ def bench_ours(args):
             out["e2e"] = e2e
         if refine:
             out["refine"] = refine
+        if two_d:
+            out["gptq2d"] = two_d
         if not args.no_cpu_baseline and world == 1:
             out["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
         print(json.dumps(out))

@@ -17,6 +17,9 @@ recipes reproduce their shapes and spectral structure:
                 power-law spectrum (exp -1.2)
 * ``lowrank``   W as ``mlp_down``; X = rank-64 signal at 100x the energy of an
                 isotropic N(0, 1) noise floor
+* ``two_sided`` two-sided rounding problem on the ``mlp_down`` shape: X 2048x6144 fp32
+                ~ N(0, 9) (weights in grid steps), G 2048x2048 and H 6144x6144 fp32 Gram
+                matrices Q diag(l) Q^T, Q Haar, l a power law (exponent 1, mean 1) + 0.01
 
 Every draw comes from a ``torch.Generator`` seeded from (seed, stream id,
 chunk index); calibration rows are produced in chunks of 16384 tokens so the
@@ -32,7 +35,7 @@ import torch
 CHUNK_TOKENS = 16384
 
 # Stream ids keep the draws for different tensors of one layer independent.
-_S_W, _S_BASIS, _S_X, _S_OUTLIER, _S_SPIKE, _S_SIGNAL = range(6)
+_S_W, _S_BASIS, _S_X, _S_OUTLIER, _S_SPIKE, _S_SIGNAL, _S_G2D, _S_H2D = range(8)
 
 
 def _gen(seed: int, stream: int, chunk: int, device) -> torch.Generator:
@@ -208,3 +211,28 @@ WORKLOADS = {
     "deit_fc2": lambda **kw: deit("fc2", **kw),
     "lowrank": lowrank,
 }
+
+
+@dataclass
+class TwoSided:
+    """A two-sided rounding problem: X (m x n) and the Gram matrices G (m x m), H (n x n)."""
+    name: str
+    X: torch.Tensor
+    G: torch.Tensor
+    H: torch.Tensor
+
+
+def spectral_gram(k, alpha, floor, seed, stream, device) -> torch.Tensor:
+    """Q diag(l) Q^T in fp32 (symmetrised in fp64), Q Haar, l = power law (mean 1) + floor."""
+    Q = random_orthogonal(k, k, seed, stream, device).double()
+    lam = power_law(k, alpha, device).double() + floor
+    M = (Q * lam) @ Q.t()
+    return ((M + M.t()) * 0.5).float().contiguous()
+
+
+def two_sided(m=2048, n=6144, device="cpu", seed=5, x_std=3.0, alpha=1.0, floor=0.01) -> TwoSided:
+    g = _gen(seed, _S_X, 0, device)
+    X = torch.randn(m, n, generator=g, device=device) * x_std
+    G = spectral_gram(m, alpha, floor, seed, _S_G2D, device)
+    H = spectral_gram(n, alpha, floor, seed, _S_H2D, device)
+    return TwoSided(f"two-sided {m}x{n}", X.contiguous(), G, H)

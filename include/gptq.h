@@ -10,6 +10,7 @@
  *   gptq_il_quantize_layer    the same pass on the augmented calibration [X, X V_r]; returns Q, L = V_r, R
  *   gptq_il_refine            OLrC + Bid-Up refinement rounds on a quantized layer: new L, R, codes
  *   gptq_quantize_lowrank     L and R stored at low precision (4-bit L, 8-bit R) on min-max grids
+ *   gptq_2d_round             two-sided adaptive rounding of a real matrix to integers (GPTQ-2D)
  *
  * Conventions shared by every entry point
  *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);
@@ -64,7 +65,8 @@ typedef enum {
     GPTQ_OP_PREPARE_HINV = 1,
     GPTQ_OP_QUANTIZE = 2,
     GPTQ_OP_IL_QUANTIZE = 3,
-    GPTQ_OP_IL_REFINE = 4
+    GPTQ_OP_IL_REFINE = 4,
+    GPTQ_OP_2D_ROUND = 5
 } gptq_op;
 
 /* Bytes of device workspace the entry point `op` needs for these sizes (0 if none).
@@ -263,6 +265,36 @@ GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, in
                                    int bits_L, int group_size_L, int bits_R, uint32_t *codes_L,
                                    float *scales_L, uint8_t *zeros_L, uint32_t *codes_R,
                                    float *scales_R, uint8_t *zeros_R, gptq_stream_t stream);
+
+/*
+ * gptq_2d_round — two-sided adaptive rounding (GPTQ-2D: Cubic-Time Two-Sided Adaptive
+ * Rounding, sections 1-2).
+ *
+ * Finds integers Z for the real matrix X that approximately minimise ||A (Z - X) B||_F^2
+ * given the Gram matrices G = A^T A (m x m) and H = B B^T (n x n): the one-sided adaptive
+ * rounding of vec X (columns stacked) under H (x) G, run as the anti-diagonal wavefront.
+ * Entries are decided in the order of the vectorised sweep up to independence (section 3,
+ * Theorems 1 and 2), each as rint(v) with ties to even, v the entry minus the feedback of
+ * all earlier errors; there is no grid and no clipping. The feedback factors are the upper
+ * U_G, U_H with G^-1 = U_G^T U_G, H^-1 = U_H^T U_H (no damping: A and B are non-singular).
+ *
+ *   X          device fp32, m x n row-major.
+ *   m, n       0 <= m, n <= 65536; m == 0 or n == 0 is a no-op returning GPTQ_OK.
+ *   G          device fp32, m x m row-major, symmetric positive definite (upper triangle read).
+ *   H          device fp32, n x n row-major, symmetric positive definite (upper triangle read).
+ *   Z          device int32, m x n row-major, written. Values outside the int32 range
+ *              saturate in Z; the sweep itself continues with the unsaturated integer.
+ *   err        device fp32, m x n row-major, written with the errors e = (v - z) / (U_G[p,p]
+ *              U_H[q,q]) of the sweep; may be NULL.
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_2D_ROUND, m, n, 0, 0) bytes, 256-byte
+ *              aligned.
+ * Returns GPTQ_ERR_ARG (bad pointer or size) or GPTQ_ERR_WORKSPACE before enqueueing
+ * anything. Device-side: GPTQ_ERR_NOT_PD if G or H is not numerically positive definite,
+ * GPTQ_ERR_NONFINITE (info: the tile row of the entry) if a pre-rounding value is not finite.
+ */
+GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G, const float *H,
+                           int32_t *Z, float *err, void *workspace, size_t ws_bytes,
+                           gptq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -19,12 +19,12 @@ GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, -1, -2, -3
 GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
-GPTQ_OP_IL_REFINE = 4
+GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND = 4, 5
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
             "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-            "gptq_quantize_lowrank")
+            "gptq_quantize_lowrank", "gptq_2d_round")
 
 
 class GptqError(RuntimeError):
@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
                                    c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
         "gptq_quantize_lowrank": (c_int, [c_p, c_p, c_i64, c_i64, c_int, c_int, c_int, c_int,
                                           c_p, c_p, c_p, c_p, c_p, c_p, c_p]),
+        "gptq_2d_round": (c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -239,6 +240,40 @@ def gptq_quantize_lowrank(L: torch.Tensor, R: torch.Tensor, bits_L: int, group_s
                                       _ptr(codes_L), _ptr(scales_L), _ptr(zeros_L), _ptr(codes_R),
                                       _ptr(scales_R), _ptr(zeros_R), _stream(stream)),
            "gptq_quantize_lowrank")
+
+
+def gptq_2d_round(X: torch.Tensor, G: torch.Tensor, H: torch.Tensor, Z: torch.Tensor,
+                  err: torch.Tensor | None, ws: torch.Tensor | None, stream=None):
+    m, n = X.shape
+    if m and n:
+        for t, name in ((X, "X"), (G, "G"), (H, "H")):
+            _dev(t, name, torch.float32)
+        _dev(Z, "Z", torch.int32)
+        if err is not None:
+            _dev(err, "err", torch.float32)
+        if G.shape != (m, m) or H.shape != (n, n) or Z.shape != (m, n):
+            raise ValueError("gptq_2d_round: G must be m x m, H n x n, Z m x n")
+    nbytes = 0 if ws is None else ws.numel()
+    _check(_lib.gptq_2d_round(_ptr(X), m, n, _ptr(G), _ptr(H), _ptr(Z), _ptr(err), _ptr(ws),
+                              nbytes, _stream(stream)), "gptq_2d_round")
+
+
+def round_2d(X: torch.Tensor, G: torch.Tensor, H: torch.Tensor, *, with_err: bool = False,
+             check_status: bool = True) -> dict:
+    """Two-sided adaptive rounding of X (m x n) under G (m x m) and H (n x n) with fresh
+    outputs: Z (int32) and, if asked, the errors."""
+    m, n = X.shape
+    dev = X.device
+    Z = torch.empty(m, n, dtype=torch.int32, device=dev)
+    err = torch.empty(m, n, dtype=torch.float32, device=dev) if with_err else None
+    ws = workspace(GPTQ_OP_2D_ROUND, m, n, 0, 0, dev) if m and n else None
+    gptq_2d_round(X, G, H, Z, err, ws)
+    if check_status:
+        gptq_sync_status()
+    out = dict(Z=Z)
+    if with_err:
+        out["err"] = err
+    return out
 
 
 # ------------------------------------------------------------------------------------------

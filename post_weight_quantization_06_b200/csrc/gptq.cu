@@ -9,6 +9,7 @@
 #include "quant.cuh"
 #include "il.cuh"
 #include "refine.cuh"
+#include "gptq2d.cuh"
 #include "hessian_tc.cuh"
 
 namespace gptq {
@@ -93,6 +94,27 @@ inline RefineWs carve_refine(Carver &c, long long m, long long n, int r) {
     w.rowloss = c.take<double>((size_t)m);
     if (r > 0) w.il = carve_ilwork(c, m, r);
     else std::memset(&w.il, 0, sizeof(w.il));
+    return w;
+}
+
+struct TwoDWs {
+    FactorWs f;
+    float *UG, *UH, *Xw, *Cacc, *E, *F, *lam;
+    long long Mp, Np;
+};
+// Factors and tile buffers of gptq_2d_round, on the shapes padded to whole 32 x 32 tiles.
+inline TwoDWs carve_2d(Carver &c, long long m, long long n) {
+    TwoDWs w;
+    w.Mp = (m + T2D - 1) / T2D * T2D;
+    w.Np = (n + T2D - 1) / T2D * T2D;
+    w.f = carve_factor(c, m > n ? m : n);
+    w.UG = c.take<float>((size_t)(w.Mp * w.Mp));
+    w.UH = c.take<float>((size_t)(w.Np * w.Np));
+    w.Xw = c.take<float>((size_t)(w.Mp * w.Np));
+    w.Cacc = c.take<float>((size_t)(w.Mp * w.Np));
+    w.E = c.take<float>((size_t)(w.Mp * w.Np));
+    w.F = c.take<float>((size_t)(w.Mp * w.Np));
+    w.lam = c.take<float>(1);
     return w;
 }
 
@@ -215,6 +237,10 @@ GPTQ_API size_t gptq_workspace_size(int op, int64_t m, int64_t n, int r, int blo
         case GPTQ_OP_IL_REFINE:
             if (m < 1 || r < 0) return 0;
             carve_refine(c, m, n, r);
+            return c.off;
+        case GPTQ_OP_2D_ROUND:
+            if (m < 1 || m > 65536 || n > 65536) return 0;
+            carve_2d(c, m, n);
             return c.off;
         default:
             return 0;
@@ -408,6 +434,37 @@ GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, in
     rtn_rows_kernel<<<ceil_div(m, 8), 256, 0, s>>>(R, 1, m, (int)m, r, bits_R, r, codes_R,
                                                    (long long)r * bits_R / 32, scales_R, zeros_R, 1);
     return launch_status();
+}
+
+GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G, const float *H,
+                           int32_t *Z, float *err, void *workspace, size_t ws_bytes,
+                           gptq_stream_t stream) {
+    if (m < 0 || n < 0 || m > 65536 || n > 65536) return GPTQ_ERR_ARG;
+    if (m == 0 || n == 0) return GPTQ_OK;
+    if (!X || !G || !H || !Z) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_2D_ROUND, m, n, 0, 0);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(workspace);
+    TwoDWs w = carve_2d(c, m, n);
+    // U_G, U_H (no damping), identity rows on the padding
+    if (int st = prepare_hinv_impl(G, (int)m, 0.f, w.UG, w.Mp, w.lam, w.f, s)) return st;
+    if (w.Mp > m) {
+        gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(w.UG, m, w.Mp);
+        GPTQ_CHECK_LAUNCH();
+    }
+    if (int st = prepare_hinv_impl(H, (int)n, 0.f, w.UH, w.Np, w.lam, w.f, s)) return st;
+    if (w.Np > n) {
+        gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(w.UH, n, w.Np);
+        GPTQ_CHECK_LAUNCH();
+    }
+    gptq2d_init_kernel<<<1184, 256, 0, s>>>(X, (int)m, (int)n, w.Xw, w.Cacc, w.Mp, w.Np);
+    GPTQ_CHECK_LAUNCH();
+    Gptq2dArgs a;
+    a.Xw = w.Xw; a.Cacc = w.Cacc; a.E = w.E; a.F = w.F; a.UG = w.UG; a.UH = w.UH;
+    a.Z = Z; a.err = err; a.Mp = w.Mp; a.Np = w.Np; a.m = (int)m; a.n = (int)n;
+    a.MT = (int)(w.Mp / T2D); a.NT = (int)(w.Np / T2D);
+    return gptq2d_sweep(a, s);
 }
 
 }  // extern "C"

@@ -21,7 +21,7 @@ def test_header_declares_the_boundary():
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
         "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-        "gptq_quantize_lowrank"])
+        "gptq_quantize_lowrank", "gptq_2d_round"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -65,7 +65,12 @@ def test_workspace_sizes():
     assert rf >= 3 * 2048 * 6144 * 4 + 2048 * 2048 * 4
     assert g.gptq_workspace_size(g.GPTQ_OP_IL_REFINE, 2048, 6144, 0, 0) < rf
     assert g.gptq_workspace_size(99, 1, 1) == 0
-    for v in (f, q, il0, il, rf):
+    t2 = g.gptq_workspace_size(g.GPTQ_OP_2D_ROUND, 2048, 6144)
+    assert t2 >= (2 * 6144 * 6144 + 2048 * 2048 + 4 * 2048 * 6144) * 4
+    # ragged shapes are padded to whole 32 x 32 tiles
+    assert g.gptq_workspace_size(g.GPTQ_OP_2D_ROUND, 70, 100) >= (2 * 128 * 128 + 96 * 96 + 4 * 96 * 128) * 4
+    assert g.gptq_workspace_size(g.GPTQ_OP_2D_ROUND, 0, 100) == 0
+    for v in (f, q, il0, il, rf, t2):
         assert v % 256 == 0
 
 
@@ -164,3 +169,24 @@ def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     monkeypatch.setattr(g, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         g._load()
+
+
+@pytest.mark.parametrize("X,m,n,G,H,Z", [(NULL, 8, 8, P, P, P), (P, 8, 8, NULL, P, P),
+                                         (P, 8, 8, P, NULL, P), (P, 8, 8, P, P, NULL),
+                                         (P, -1, 8, P, P, P), (P, 8, -3, P, P, P),
+                                         (P, 65537, 8, P, P, P), (P, 8, 70000, P, P, P)])
+def test_2d_round_rejects_bad_arguments(X, m, n, G, H, Z):
+    st = _lib().gptq_2d_round(X, m, n, G, H, Z, NULL, ctypes.c_void_p(1 << 20), 1 << 40, NULL)
+    assert st == -1
+
+
+def test_2d_round_checks_the_workspace_and_accepts_empty_input():
+    import post_weight_quantization_06_b200 as g
+    need = g.gptq_workspace_size(g.GPTQ_OP_2D_ROUND, 40, 70)
+    lib = _lib()
+    assert lib.gptq_2d_round(P, 40, 70, P, P, P, NULL, ctypes.c_void_p(1 << 20), need - 256, NULL) == -6
+    assert lib.gptq_2d_round(P, 40, 70, P, P, P, NULL, ctypes.c_void_p((1 << 20) + 16), need, NULL) == -6
+    assert lib.gptq_2d_round(P, 40, 70, P, P, P, NULL, NULL, need, NULL) == -6
+    # nothing to round: returns at once, touching no pointer
+    assert lib.gptq_2d_round(NULL, 0, 70, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
+    assert lib.gptq_2d_round(NULL, 40, 0, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0

@@ -364,13 +364,16 @@ struct FactorStreams {
     bool ready = false;
 };
 
-inline FactorStreams *factor_streams() {
-    static FactorStreams fs[64];
+// One set per device and slot: factorizations enqueued on different slots can run at once.
+constexpr int FACTOR_SLOTS = 2;
+inline FactorStreams *factor_streams(int slot) {
+    static FactorStreams fs[64][FACTOR_SLOTS];
     static std::mutex init_mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (slot < 0 || slot >= FACTOR_SLOTS) return nullptr;
     std::lock_guard<std::mutex> lk(init_mu);
-    FactorStreams &f = fs[dev];
+    FactorStreams &f = fs[dev][slot];
     if (!f.ready) {
         int lo = 0, hi = 0;
         cudaDeviceGetStreamPriorityRange(&lo, &hi);
@@ -401,9 +404,9 @@ inline FactorStreams *factor_streams() {
 // over the finished row blocks l, from Ubar X = I. The chain waits for the bulk update of
 // the previous block before its look-ahead; the inverse stream trails both.
 inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n, float *T,
-                             cudaStream_t s) {
+                             cudaStream_t s, int slot = 0) {
     if (n <= FACTOR_NB) return leaf_ul_inv(A, lda, U, ldu, n, 0, s);
-    FactorStreams *fs = factor_streams();
+    FactorStreams *fs = factor_streams(slot);
     if (!fs) return GPTQ_ERR_CUDA;
     std::lock_guard<std::mutex> lk(fs->mu);
     int dev = 0, sms = 148;

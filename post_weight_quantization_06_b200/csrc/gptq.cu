@@ -98,7 +98,7 @@ inline RefineWs carve_refine(Carver &c, long long m, long long n, int r) {
 }
 
 struct TwoDWs {
-    FactorWs f;
+    FactorWs fg, fh;
     float *UG, *UH, *Xw, *Cacc, *E, *F, *lam;
     long long Mp, Np;
 };
@@ -107,14 +107,15 @@ inline TwoDWs carve_2d(Carver &c, long long m, long long n) {
     TwoDWs w;
     w.Mp = (m + T2D - 1) / T2D * T2D;
     w.Np = (n + T2D - 1) / T2D * T2D;
-    w.f = carve_factor(c, m > n ? m : n);
+    w.fg = carve_factor(c, m);
+    w.fh = carve_factor(c, n);
     w.UG = c.take<float>((size_t)(w.Mp * w.Mp));
     w.UH = c.take<float>((size_t)(w.Np * w.Np));
     w.Xw = c.take<float>((size_t)(w.Mp * w.Np));
     w.Cacc = c.take<float>((size_t)(w.Mp * w.Np));
     w.E = c.take<float>((size_t)(w.Mp * w.Np));
     w.F = c.take<float>((size_t)(w.Mp * w.Np));
-    w.lam = c.take<float>(1);
+    w.lam = c.take<float>(2);
     return w;
 }
 
@@ -166,13 +167,13 @@ int hessian_simt(float *H, const TX *X, long long k, int n, cudaStream_t s) {
 }
 
 int prepare_hinv_impl(const float *H, int n, float lambda_rel, float *U, long long ldu,
-                      float *lambda_out, FactorWs &w, cudaStream_t s) {
+                      float *lambda_out, FactorWs &w, cudaStream_t s, int slot = 0) {
     damp_mean_kernel<<<1, 1024, 0, s>>>(H, n, n, lambda_rel, lambda_out);
     GPTQ_CHECK_LAUNCH();
     copy_damped_kernel<<<1184, 256, 0, s>>>(H, n, w.A, n, n, lambda_out);
     GPTQ_CHECK_LAUNCH();
     if (cudaMemsetAsync(U, 0, sizeof(float) * (size_t)n * ldu, s) != cudaSuccess) return GPTQ_ERR_CUDA;
-    return factor_ul_inverse(w.A, n, U, ldu, n, w.T, s);
+    return factor_ul_inverse(w.A, n, U, ldu, n, w.T, s, slot);
 }
 
 int init_work(const void *W, int w_dtype, long long m, int n, float *Wc, long long ldw, int N,
@@ -447,16 +448,28 @@ GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     Carver c(workspace);
     TwoDWs w = carve_2d(c, m, n);
-    // U_G, U_H (no damping), identity rows on the padding
-    if (int st = prepare_hinv_impl(G, (int)m, 0.f, w.UG, w.Mp, w.lam, w.f, s)) return st;
-    if (w.Mp > m) {
-        gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(w.UG, m, w.Mp);
-        GPTQ_CHECK_LAUNCH();
-    }
-    if (int st = prepare_hinv_impl(H, (int)n, 0.f, w.UH, w.Np, w.lam, w.f, s)) return st;
-    if (w.Np > n) {
-        gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(w.UH, n, w.Np);
-        GPTQ_CHECK_LAUNCH();
+    // U_G (side stream, second factor slot) and U_H (this stream) at once, no damping;
+    // identity rows on the padding
+    Gptq2dSide *side = gptq2d_side();
+    if (!side) return GPTQ_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(side->mu);
+        if (cudaEventRecord(side->fork, s) != cudaSuccess ||
+            cudaStreamWaitEvent(side->stream, side->fork, 0) != cudaSuccess)
+            return GPTQ_ERR_CUDA;
+        if (int st = prepare_hinv_impl(G, (int)m, 0.f, w.UG, w.Mp, w.lam + 1, w.fg, side->stream, 1))
+            return st;
+        if (w.Mp > m) {
+            gptq2d_pad_identity_kernel<<<64, 256, 0, side->stream>>>(w.UG, m, w.Mp);
+            GPTQ_CHECK_LAUNCH();
+        }
+        if (cudaEventRecord(side->join, side->stream) != cudaSuccess) return GPTQ_ERR_CUDA;
+        if (int st = prepare_hinv_impl(H, (int)n, 0.f, w.UH, w.Np, w.lam, w.fh, s, 0)) return st;
+        if (w.Np > n) {
+            gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(w.UH, n, w.Np);
+            GPTQ_CHECK_LAUNCH();
+        }
+        if (cudaStreamWaitEvent(s, side->join, 0) != cudaSuccess) return GPTQ_ERR_CUDA;
     }
     gptq2d_init_kernel<<<1184, 256, 0, s>>>(X, (int)m, (int)n, w.Xw, w.Cacc, w.Mp, w.Np);
     GPTQ_CHECK_LAUNCH();

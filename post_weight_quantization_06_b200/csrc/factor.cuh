@@ -340,11 +340,217 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_ul_inv_kernel(const float *
     }
 }
 
+// ---------------------------------------------------------------------------------------
+// Leaf of the blocked factor, itself blocked (fp32): the 128 x 128 block is cut into four
+// 32-column blocks, last first, and for block k (columns r .. r + 31) of the Schur
+// complement S (shared memory, both triangles kept):
+//   A  one warp: UL-Cholesky of S[k, k] and the inverse X_kk of its factor, in registers
+//      (lane i holds row i; the column sweep of the barrier leaf, with its row and column
+//      exchanged through shared memory inside the warp);
+//   B  Ubar's panel Ubar[0:r, k] = S[0:r, k] X_kk^T, written over S[0:r, k];
+//   C  S[0:r, 0:r] -= Ubar[0:r, k] Ubar[0:r, k]^T;
+//   D  X[k, >k] = -X_kk (Ubar[k, >k] X[>k, >k]): the inverse's rows right of the diagonal.
+// A block with nb < 128 is padded with the identity (it couples to nothing). Only the
+// diagonal steps of A are sequential; B, C and D are small products over all 8 warps.
+// ---------------------------------------------------------------------------------------
+constexpr int LB = 32;
+constexpr int LB_LD = FACTOR_NB + 1;     // padded stride of S and X
+constexpr int LB_TLD = FACTOR_NB - LB + 1;
+constexpr size_t LEAF_BLK_SMEM =
+    sizeof(float) * (2 * (size_t)FACTOR_NB * LB_LD + (size_t)LB * LB_TLD + 4 * LB);
+
+__global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, long long lda,
+                                                                float *U, long long ldu, int nb,
+                                                                long long col_base) {
+    extern __shared__ __align__(16) float lsm[];
+    float *Sm = lsm;                                  // [128][129] Schur complement / panels
+    float *Xm = Sm + FACTOR_NB * LB_LD;               // [128][129] the inverse (upper)
+    float *Tm = Xm + FACTOR_NB * LB_LD;               // [32][97]   Ubar[k, >k] X[>k, >k]
+    float *xb = Tm + LB * LB_TLD;                     // [2][2][32] step exchange (u, row c)
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+
+#pragma unroll 4
+    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
+        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
+        float v;
+        if (i < nb && j < nb) v = j >= i ? A[(long long)i * lda + j] : A[(long long)j * lda + i];
+        else v = i == j ? 1.f : 0.f;
+        Sm[i * LB_LD + j] = v;
+        Xm[i * LB_LD + j] = 0.f;
+    }
+    __syncthreads();
+
+#pragma unroll 1
+    for (int kb = FACTOR_NB / LB - 1; kb >= 0; --kb) {
+        const int r = kb * LB;
+        const int q = FACTOR_NB - r - LB;             // columns right of block k
+        // ---- A: the diagonal block -------------------------------------------------------
+        if (w == 0) {
+            const int i = lane;
+            float m[LB];
+#pragma unroll
+            for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
+#pragma unroll
+            for (int c = LB - 1; c >= 0; --c) {
+                float *ub = xb + (c & 1) * 2 * LB, *rb = ub + LB;
+                const float d = __shfl_sync(0xffffffffu, m[c], c);
+                const bool bad = !(d > 0.f) || !isfinite(d);
+                if (bad && i == 0) report(GPTQ_ERR_NOT_PD, col_base + r + c);
+                const float dd = bad ? 1.f : d;
+                float ip = rsqrtf(dd);
+                ip = ip * (1.5f - 0.5f * dd * ip * ip);  // one Newton step
+                const float u = i < c ? m[c] * ip : 0.f;
+                ub[i] = -u;
+                if (i == c) {
+#pragma unroll
+                    for (int j = c + 1; j < LB; ++j) rb[j] = -ip * m[j];
+                }
+                __syncwarp();
+                if (i == c) {
+                    m[c] = ip;
+#pragma unroll
+                    for (int j = c + 1; j < LB; ++j) m[j] = rb[j];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < c; ++j) m[j] = fmaf(u, ub[j], m[j]);
+                    m[c] = u * ip;
+#pragma unroll
+                    for (int j = c + 1; j < LB; ++j) m[j] = fmaf(u, rb[j], m[j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < LB; ++j) Xm[(r + i) * LB_LD + r + j] = j >= i ? m[j] : 0.f;
+        }
+        __syncthreads();
+        // ---- B (compute) and D1 ----------------------------------------------------------
+        float pb[12];
+        if (r > 0) {
+#pragma unroll
+            for (int t = 0; t < 12; ++t) pb[t] = 0.f;
+            const int c = lane;
+#pragma unroll 4
+            for (int mm = 0; mm < LB; ++mm) {
+                const float x = Xm[(r + c) * LB_LD + r + mm];
+#pragma unroll
+                for (int t = 0; t < 12; ++t)
+                    if (w + 8 * t < r) pb[t] = fmaf(Sm[(w + 8 * t) * LB_LD + r + mm], x, pb[t]);
+            }
+        }
+        if (q > 0) {
+            float acc[4][3];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < 3; ++h) acc[p][h] = 0.f;
+            for (int mm = r + LB; mm < FACTOR_NB; ++mm) {
+                float x[3], sv[4];
+#pragma unroll
+                for (int h = 0; h < 3; ++h) {
+                    const int jj = lane + 32 * h;
+                    x[h] = jj < q ? Xm[mm * LB_LD + r + LB + jj] : 0.f;
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p) sv[p] = Sm[(r + w + 8 * p) * LB_LD + mm];
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+#pragma unroll
+                    for (int h = 0; h < 3; ++h) acc[p][h] = fmaf(sv[p], x[h], acc[p][h]);
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < 3; ++h) {
+                    const int jj = lane + 32 * h;
+                    if (jj < q) Tm[(w + 8 * p) * LB_TLD + jj] = acc[p][h];
+                }
+        }
+        __syncthreads();
+        // ---- B (write) and D2 ------------------------------------------------------------
+        if (r > 0) {
+#pragma unroll
+            for (int t = 0; t < 12; ++t)
+                if (w + 8 * t < r) Sm[(w + 8 * t) * LB_LD + r + lane] = pb[t];
+        }
+        if (q > 0) {
+            float acc[4][3];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < 3; ++h) acc[p][h] = 0.f;
+#pragma unroll 4
+            for (int c2 = 0; c2 < LB; ++c2) {
+                float x[4], tv[3];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) x[p] = Xm[(r + w + 8 * p) * LB_LD + r + c2];
+#pragma unroll
+                for (int h = 0; h < 3; ++h) {
+                    const int jj = lane + 32 * h;
+                    tv[h] = jj < q ? Tm[c2 * LB_TLD + jj] : 0.f;
+                }
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+#pragma unroll
+                    for (int h = 0; h < 3; ++h) acc[p][h] = fmaf(x[p], tv[h], acc[p][h]);
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < 3; ++h) {
+                    const int jj = lane + 32 * h;
+                    if (jj < q) Xm[(r + w + 8 * p) * LB_LD + r + LB + jj] = -acc[p][h];
+                }
+        }
+        __syncthreads();
+        // ---- C: the Schur complement -----------------------------------------------------
+        if (r > 0) {
+            const int tx = tid & 15, ty = tid >> 4;
+            float acc[6][6];
+#pragma unroll
+            for (int a = 0; a < 6; ++a)
+#pragma unroll
+                for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+            for (int c = 0; c < LB; ++c) {
+                float pa[6], pbv[6];
+#pragma unroll
+                for (int a = 0; a < 6; ++a) {
+                    pa[a] = ty + 16 * a < r ? Sm[(ty + 16 * a) * LB_LD + r + c] : 0.f;
+                    pbv[a] = tx + 16 * a < r ? Sm[(tx + 16 * a) * LB_LD + r + c] : 0.f;
+                }
+#pragma unroll
+                for (int a = 0; a < 6; ++a)
+#pragma unroll
+                    for (int b = 0; b < 6; ++b) acc[a][b] = fmaf(pa[a], pbv[b], acc[a][b]);
+            }
+#pragma unroll
+            for (int a = 0; a < 6; ++a)
+#pragma unroll
+                for (int b = 0; b < 6; ++b) {
+                    const int i = ty + 16 * a, j = tx + 16 * b;
+                    if (i < r && j < r) Sm[i * LB_LD + j] -= acc[a][b];
+                }
+        }
+        __syncthreads();
+    }
+#pragma unroll 4
+    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
+        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
+        if (i < nb && j < nb) U[(long long)i * ldu + j] = j >= i ? Xm[i * LB_LD + j] : 0.f;
+    }
+}
+
 inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, int nb,
                        long long col_base, cudaStream_t s) {
-    // GPTQ_WARP_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
-    static const bool warp_leaf = tc::env_ll("GPTQ_WARP_LEAF", 1) != 0;
-    if (!warp_leaf) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
+    // GPTQ_LEAF: 0 the barrier-synchronised leaf (diag_ul_inv_kernel), 1 (default) the
+    // warp-owner leaf, 2 the blocked leaf
+    static const long long leaf = tc::env_ll("GPTQ_LEAF", 1);
+    if (leaf == 0) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
+    if (leaf == 2) {
+        cudaFuncSetAttribute(leaf_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)LEAF_BLK_SMEM);
+        leaf_blk_kernel<<<1, LEAF_THREADS, LEAF_BLK_SMEM, s>>>(A, lda, U, ldu, nb, col_base);
+        return launch_status();
+    }
     cudaFuncSetAttribute(leaf_ul_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)LEAF_SMEM);
     // clock cycles a warp waits for a step before the kernel gives up with GPTQ_ERR_TIMEOUT

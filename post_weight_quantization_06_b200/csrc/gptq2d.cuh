@@ -262,9 +262,12 @@ __global__ __launch_bounds__(T2D_THREADS) void gptq2d_sweep_kernel(Gptq2dArgs a,
                 }
                 const float2 ncf = make_float2(-cf, -cf);
 #pragma unroll
-                for (int P = 0; P < T2D / 2; ++P) {
-                    // slots 2P, 2P+1 are d0 = (2P - u) % 32 and d1 = (d0 + 1) % 32 steps ahead;
-                    // d = 0 is the slot just consumed (its weights are zero or unused)
+                for (int i = 0; i < T2D / 2; ++i) {
+                    // the pair holding the next step's slot first (the next decision waits on
+                    // it), then the rest. Slots 2P, 2P+1 are d0 = (2P - u) % 32 and d1 =
+                    // (d0 + 1) % 32 steps ahead; d = 0 is the slot just consumed (its weights
+                    // are zero or unused)
+                    const int P = (((u + 1) >> 1) + i) & (T2D / 2 - 1);
                     const int d0 = (2 * P - u) & 31, d1 = (d0 + 1) & 31;
                     const float e0 = d0 ? __shfl_up_sync(0xffffffffu, e, d0) : e;
                     const float e1 = d1 ? __shfl_up_sync(0xffffffffu, e, d1) : e;

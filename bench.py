@@ -340,6 +340,7 @@ def run_gptq2d(g, dev, steps):
     time minus H's factorization (the figure the roofline uses)."""
     import datagen
     P = datagen.two_sided(device=dev)
+    torch.cuda.synchronize(dev)           # the inputs come from the current stream
     m, n = P.X.shape
     Z = torch.empty(m, n, dtype=torch.int32, device=dev)
     ws = g.workspace(g.GPTQ_OP_2D_ROUND, m, n, 0, 0, dev)
@@ -453,6 +454,7 @@ def bench_ours(args):
     if args.tokens:
         layer.X = layer.X[: args.tokens].clone()
         torch.cuda.empty_cache()
+    torch.cuda.synchronize(dev)           # generated on the current stream, used on others
     stream = torch.cuda.Stream(device=dev)
     lp = LayerPass(g, layer, stream)
     for _ in range(args.warmup):

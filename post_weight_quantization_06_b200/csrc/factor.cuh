@@ -174,201 +174,209 @@ __global__ void copy_damped_kernel(const float *H, long long ldh, float *A, long
 }
 
 // ---------------------------------------------------------------------------------------
-// Leaf of the blocked factor (fp32): the same UL sweep as diag_ul_inv_kernel, organised so
-// that no step waits on a CTA-wide barrier. Warp w owns the 16 columns 16w..16w+15; lane l
-// holds rows l, l+32, l+64, l+96 of them (64 registers). Step c belongs to the warp that
-// owns column c: it takes the pivot, publishes u = M[:c, c] / sqrt(d) and 1/sqrt(d) to
-// shared memory (one slot per step, written once) and its 32 lanes arrive on the step's
-// mbarrier (release). Every other warp waits on that barrier (acquire; the hardware parks
-// the waiting threads) and applies the step to its own columns: the Cholesky update
-// (v_j = -u_j) left of c, the inverse update (v_j = -P[c][j] / sqrt(d), row c read from the
-// lane that holds it) right of c.
-//   Row c is final after step c (row c of the inverse, columns >= c): it goes to shared
-// memory and its registers are dead, as are all rows below it, so step c only touches the
-// row slots that still hold rows < c. During its 16 steps the owner rotates its columns by
-// one register position per step (the update of position p lands in p + 1, the restarted
-// pivot column in 0), so the pivot is always in position 15 and every register index is a
-// compile-time constant; 16 rotations restore the order. Only the loop over the 4 row slots
-// is unrolled, which keeps the code each warp runs within the instruction cache.
-// ---------------------------------------------------------------------------------------
-constexpr int LEAF_THREADS = 256;
-constexpr int LEAF_LD = FACTOR_NB + 1;  // padded stride of the staging tile
-constexpr size_t LEAF_SMEM = sizeof(float) * (2 * (size_t)FACTOR_NB * FACTOR_NB + FACTOR_NB);
-static_assert(FACTOR_NB * LEAF_LD <= 2 * FACTOR_NB * FACTOR_NB, "staging fits the step slots");
-
-template <int RC>
-__device__ __forceinline__ void leaf_rotate(float (&M)[4][16]) {
-#pragma unroll
-    for (int r = 0; r <= RC; ++r) {
-        const float t = M[r][15];
-#pragma unroll
-        for (int p = 14; p >= 0; --p) M[r][p + 1] = M[r][p];
-        M[r][0] = t;
-    }
-}
-
-// Steps c = 32 RC + 31 .. 32 RC of the sweep (rows of slot RC).
-template <int RC>
-__device__ __forceinline__ void leaf_slot_steps(float (&M)[4][16], float *pub, float *xrow,
-                                                float *pipiv, uint64_t *step_bar, int nb,
-                                                long long col_base, long long wait_limit,
-                                                int lane, int w, bool &stop) {
-#pragma unroll 1
-    for (int cc = 31; cc >= 0; --cc) {
-        const int c = 32 * RC + cc, ob = c >> 4, s = 15 - (c & 15);
-        if (stop) return;
-        if (c >= nb) {
-            if (w == ob) leaf_rotate<RC>(M);  // keep the owner's rotation count
-            continue;
-        }
-        float u[RC + 1], v[16];
-        if (w == ob) {
-            const float d = __shfl_sync(0xffffffffu, M[RC][15], cc);
-            const bool bad = !(d > 0.f) || !isfinite(d);
-            if (bad && lane == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
-            const float dd = bad ? 1.f : d;
-            float ipiv = rsqrtf(dd);
-            ipiv = ipiv * (1.5f - 0.5f * dd * ipiv * ipiv);  // one Newton step
-#pragma unroll
-            for (int r = 0; r <= RC; ++r) {
-                u[r] = (r < RC || lane < cc) ? M[r][15] * ipiv : 0.f;
-                pub[c * FACTOR_NB + lane + 32 * r] = u[r];
-            }
-            if (lane == 0) pipiv[c] = ipiv;
-            tc::mbar_arrive(&step_bar[c]);
-            // position p holds column 16 ob + ((p - s) mod 16): p < s right of c, s <= p < 15
-            // left of c (its u sits in lane (16 ob + p - s) mod 32 of this slot)
-            const int jl = (16 * ob - s) & 31;
-#pragma unroll
-            for (int p = 0; p < 15; ++p) {
-                const float a = __shfl_sync(0xffffffffu, M[RC][p], cc);
-                const float b = __shfl_sync(0xffffffffu, u[RC], (jl + p) & 31);
-                v[p] = p < s ? -ipiv * a : -b;
-            }
-            v[15] = ipiv;
-            if (lane == cc) {
-#pragma unroll
-                for (int p = 0; p < 16; ++p)
-                    if (p < s || p == 15) xrow[c * FACTOR_NB + 16 * ob + ((p - s) & 15)] = v[p];
-            }
-#pragma unroll
-            for (int r = 0; r <= RC; ++r) {
-#pragma unroll
-                for (int p = 14; p >= 0; --p) M[r][p + 1] = fmaf(u[r], v[p], M[r][p]);
-                M[r][0] = u[r] * ipiv;
-            }
-        } else {
-            if (!tc::mbar_wait(&step_bar[c], 0u, wait_limit)) {
-                if (lane == 0) report(GPTQ_ERR_TIMEOUT, col_base + c);
-                stop = true;
-                return;
-            }
-            const float ipiv = pipiv[c];
-#pragma unroll
-            for (int r = 0; r <= RC; ++r) u[r] = pub[c * FACTOR_NB + lane + 32 * r];
-            if (w < ob) {
-                const float4 *q = reinterpret_cast<const float4 *>(pub + c * FACTOR_NB + 16 * w);
-#pragma unroll
-                for (int b4 = 0; b4 < 4; ++b4) {
-                    const float4 x = q[b4];
-                    v[4 * b4 + 0] = -x.x; v[4 * b4 + 1] = -x.y;
-                    v[4 * b4 + 2] = -x.z; v[4 * b4 + 3] = -x.w;
-                }
-            } else {
-#pragma unroll
-                for (int b = 0; b < 16; ++b) v[b] = -ipiv * __shfl_sync(0xffffffffu, M[RC][b], cc);
-                if (lane == cc) {
-                    float4 *q = reinterpret_cast<float4 *>(xrow + c * FACTOR_NB + 16 * w);
-#pragma unroll
-                    for (int b4 = 0; b4 < 4; ++b4)
-                        q[b4] = make_float4(v[4 * b4], v[4 * b4 + 1], v[4 * b4 + 2], v[4 * b4 + 3]);
-                }
-            }
-#pragma unroll
-            for (int r = 0; r <= RC; ++r)
-#pragma unroll
-                for (int b = 0; b < 16; ++b) M[r][b] = fmaf(u[r], v[b], M[r][b]);
-        }
-    }
-}
-
-__global__ __launch_bounds__(LEAF_THREADS) void leaf_ul_inv_kernel(const float *A, long long lda,
-                                                                   float *U, long long ldu, int nb,
-                                                                   long long col_base,
-                                                                   long long wait_limit) {
-    extern __shared__ __align__(16) float leaf_sm[];
-    float *stage = leaf_sm;                              // [128][LEAF_LD], before the sweep
-    float *pub = leaf_sm;                                // [128][128]: u of step c at pub[128 c]
-    float *xrow = leaf_sm + FACTOR_NB * FACTOR_NB;       // [128][128]: rows of the inverse
-    float *pipiv = leaf_sm + 2 * FACTOR_NB * FACTOR_NB;  // [128]
-    __shared__ uint64_t step_bar[FACTOR_NB];             // one single-use barrier per step
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-
-    // stage the block symmetrically from its upper triangle (coalesced rows)
-#pragma unroll 8
-    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
-        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
-        const float v = (j >= i && i < nb && j < nb) ? A[(long long)i * lda + j] : 0.f;
-        if (j >= i) {
-            stage[i * LEAF_LD + j] = v;
-            stage[j * LEAF_LD + i] = v;
-        }
-    }
-    if (tid < FACTOR_NB) tc::mbar_init(&step_bar[tid], 32);
-    __syncthreads();
-    float M[4][16];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int b = 0; b < 16; ++b) M[r][b] = stage[(lane + 32 * r) * LEAF_LD + 16 * w + b];
-    __syncthreads();
-
-    bool stop = false;
-    leaf_slot_steps<3>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
-                       stop);
-    leaf_slot_steps<2>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
-                       stop);
-    leaf_slot_steps<1>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
-                       stop);
-    leaf_slot_steps<0>(M, pub, xrow, pipiv, step_bar, nb, col_base, wait_limit, lane, w,
-                       stop);
-    __syncthreads();
-#pragma unroll 8
-    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
-        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
-        if (i < nb && j < nb) U[(long long)i * ldu + j] = j >= i ? xrow[i * FACTOR_NB + j] : 0.f;
-    }
-}
-
-// ---------------------------------------------------------------------------------------
 // Leaf of the blocked factor, itself blocked (fp32): the 128 x 128 block is cut into four
 // 32-column blocks, last first, and for block k (columns r .. r + 31) of the Schur
 // complement S (shared memory, both triangles kept):
 //   A  one warp: UL-Cholesky of S[k, k] and the inverse X_kk of its factor, in registers
-//      (lane i holds row i; the column sweep of the barrier leaf, with its row and column
-//      exchanged through shared memory inside the warp);
+//      (lane i holds row i). Step c needs the pivot column u = S[:c, c] / sqrt(d) and row c:
+//      while the leading block is symmetric, row c also carries the pivot column
+//      (S[c, j] = S[j, c] for j < c), so lane c's row is the only thing exchanged (one
+//      shared-memory row per step) and every lane applies m_j += a r_j with one scalar a
+//      (-u_i / sqrt(d) for rows above c, -1 - 1/sqrt(d) for row c itself, which turns its
+//      entries right of c into row c of the inverse, 0 below). Registers rotate by 4 every
+//      4 steps so the pivot's register index is static while the loop stays short;
 //   B  Ubar's panel Ubar[0:r, k] = S[0:r, k] X_kk^T, written over S[0:r, k];
 //   C  S[0:r, 0:r] -= Ubar[0:r, k] Ubar[0:r, k]^T;
 //   D  X[k, >k] = -X_kk (Ubar[k, >k] X[>k, >k]): the inverse's rows right of the diagonal.
-// A block with nb < 128 is padded with the identity (it couples to nothing). Only the
-// diagonal steps of A are sequential; B, C and D are small products over all 8 warps.
+// A block with nb < 128 is padded with the identity (it couples to nothing).
 // ---------------------------------------------------------------------------------------
 constexpr int LB = 32;
-constexpr int LB_LD = FACTOR_NB + 1;     // padded stride of S and X
-constexpr int LB_TLD = FACTOR_NB - LB + 1;
+constexpr int LB_LD = FACTOR_NB + 4;     // stride of S and X (16-byte rows)
+constexpr int LB_TLD = FACTOR_NB - LB + 4;
+constexpr int LEAF_THREADS = 256;
 constexpr size_t LEAF_BLK_SMEM =
-    sizeof(float) * (2 * (size_t)FACTOR_NB * LB_LD + (size_t)LB * LB_TLD + 4 * LB);
+    sizeof(float) * (2 * (size_t)FACTOR_NB * LB_LD + (size_t)LB * LB_TLD + 2 * LB);
+
+template <int R>
+__device__ __forceinline__ void rotate_right(float (&x)[LB]) {
+    float t[R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) t[k] = x[LB - R + k];
+#pragma unroll
+    for (int k = LB - 1; k >= R; --k) x[k] = x[k - R];
+#pragma unroll
+    for (int k = 0; k < R; ++k) x[k] = t[k];
+}
+
+// A: X_kk of the 32 x 32 block of S at (r, r), written to X (warp 0 only).
+__device__ __forceinline__ void leaf_diag32(float *Sm, float *Xm, float *rowbuf, int r,
+                                            long long col_base, int i) {
+    float m[LB];
+#pragma unroll
+    for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
+    // physical register p holds column (p - 31 + c0) mod 32 while steps c0 .. c0 - 3 run
+#pragma unroll 1
+    for (int c0 = LB - 1; c0 >= 0; c0 -= 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int c = c0 - u, P = LB - 1 - u;
+            float *rb = rowbuf + (u & 1) * LB;
+            if (i == c) {
+#pragma unroll
+                for (int p4 = 0; p4 < LB; p4 += 4)
+                    *reinterpret_cast<float4 *>(rb + p4) = make_float4(m[p4], m[p4 + 1], m[p4 + 2], m[p4 + 3]);
+            }
+            const float d = __shfl_sync(0xffffffffu, m[P], c);
+            const bool bad = !(d > 0.f) || !isfinite(d);
+            if (bad && i == 0) report(GPTQ_ERR_NOT_PD, col_base + r + c);
+            const float dd = bad ? 1.f : d;
+            float ip = rsqrtf(dd);
+            ip = ip * (1.5f - 0.5f * dd * ip * ip);  // one Newton step
+            const float uu = m[P] * ip;
+            const float a = i < c ? -uu * ip : (i == c ? -1.f - ip : 0.f);
+            __syncwarp();
+            float rv[LB];
+#pragma unroll
+            for (int p4 = 0; p4 < LB; p4 += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(rb + p4);
+                rv[p4] = t4.x; rv[p4 + 1] = t4.y; rv[p4 + 2] = t4.z; rv[p4 + 3] = t4.w;
+            }
+#pragma unroll
+            for (int p = 0; p < LB; ++p)
+                if (p != P) m[p] = fmaf(a, rv[p], m[p]);
+            m[P] = i < c ? uu * ip : ip;
+        }
+        rotate_right<4>(m);
+    }
+#pragma unroll
+    for (int j = 0; j < LB; ++j) Xm[(r + i) * LB_LD + r + j] = j >= i ? m[j] : 0.f;
+}
+
+// B, C, D of block KB (r = 32 KB rows above it, q = 96 - r columns right of it), 8 warps.
+template <int KB>
+__device__ __forceinline__ void leaf_block_updates(float *Sm, float *Xm, float *Tm, int tid) {
+    constexpr int r = KB * LB, q = FACTOR_NB - r - LB;
+    const int lane = tid & 31, w = tid >> 5;
+    // B (compute): rows w + 8 t of S[0:r, k] X_kk^T, column lane; D1: T = Ubar[k, >k] X[>k, >k]
+    constexpr int BT = r / 8;
+    float pb[BT > 0 ? BT : 1];
+    if constexpr (r > 0) {
+#pragma unroll
+        for (int t = 0; t < BT; ++t) pb[t] = 0.f;
+#pragma unroll 2
+        for (int mm = 0; mm < LB; mm += 4) {
+            const float4 x = *reinterpret_cast<const float4 *>(Xm + (r + lane) * LB_LD + r + mm);
+#pragma unroll
+            for (int t = 0; t < BT; ++t) {
+                const float4 sv = *reinterpret_cast<const float4 *>(Sm + (w + 8 * t) * LB_LD + r + mm);
+                pb[t] += sv.x * x.x + sv.y * x.y + sv.z * x.z + sv.w * x.w;
+            }
+        }
+    }
+    if constexpr (q > 0) {
+        constexpr int QH = q / 32;
+        float acc[4][QH];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int h = 0; h < QH; ++h) acc[p][h] = 0.f;
+#pragma unroll 4
+        for (int mm = r + LB; mm < FACTOR_NB; ++mm) {
+            float x[QH], sv[4];
+#pragma unroll
+            for (int h = 0; h < QH; ++h) x[h] = Xm[mm * LB_LD + r + LB + lane + 32 * h];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) sv[p] = Sm[(r + w + 8 * p) * LB_LD + mm];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < QH; ++h) acc[p][h] = fmaf(sv[p], x[h], acc[p][h]);
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int h = 0; h < QH; ++h) Tm[(w + 8 * p) * LB_TLD + lane + 32 * h] = acc[p][h];
+    }
+    __syncthreads();
+    // B (write) and D2: X[k, >k] = -X_kk T
+    if constexpr (r > 0) {
+#pragma unroll
+        for (int t = 0; t < BT; ++t) Sm[(w + 8 * t) * LB_LD + r + lane] = pb[t];
+    }
+    if constexpr (q > 0) {
+        constexpr int QH = q / 32;
+        float acc[4][QH];
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int h = 0; h < QH; ++h) acc[p][h] = 0.f;
+#pragma unroll 4
+        for (int c2 = 0; c2 < LB; ++c2) {
+            float x[4], tv[QH];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) x[p] = Xm[(r + w + 8 * p) * LB_LD + r + c2];
+#pragma unroll
+            for (int h = 0; h < QH; ++h) tv[h] = Tm[c2 * LB_TLD + lane + 32 * h];
+#pragma unroll
+            for (int p = 0; p < 4; ++p)
+#pragma unroll
+                for (int h = 0; h < QH; ++h) acc[p][h] = fmaf(x[p], tv[h], acc[p][h]);
+        }
+#pragma unroll
+        for (int p = 0; p < 4; ++p)
+#pragma unroll
+            for (int h = 0; h < QH; ++h) Xm[(r + w + 8 * p) * LB_LD + r + LB + lane + 32 * h] = -acc[p][h];
+    }
+    __syncthreads();
+    // C: S[0:r, 0:r] -= P P^T, P = S[0:r, r:r+32]; thread (ty, tx) of 16 x 16 owns rows
+    // ty + 16 a, columns tx + 16 b
+    if constexpr (r > 0) {
+        constexpr int CT = r / 16;
+        const int tx = tid & 15, ty = tid >> 4;
+        float acc[CT][CT];
+#pragma unroll
+        for (int a = 0; a < CT; ++a)
+#pragma unroll
+            for (int b = 0; b < CT; ++b) acc[a][b] = 0.f;
+#pragma unroll 2
+        for (int c = 0; c < LB; c += 4) {
+            float4 pa[CT], pv[CT];
+#pragma unroll
+            for (int a = 0; a < CT; ++a) {
+                pa[a] = *reinterpret_cast<const float4 *>(Sm + (ty + 16 * a) * LB_LD + r + c);
+                pv[a] = *reinterpret_cast<const float4 *>(Sm + (tx + 16 * a) * LB_LD + r + c);
+            }
+#pragma unroll
+            for (int a = 0; a < CT; ++a)
+#pragma unroll
+                for (int b = 0; b < CT; ++b)
+                    acc[a][b] += pa[a].x * pv[b].x + pa[a].y * pv[b].y + pa[a].z * pv[b].z + pa[a].w * pv[b].w;
+        }
+#pragma unroll
+        for (int a = 0; a < CT; ++a)
+#pragma unroll
+            for (int b = 0; b < CT; ++b) Sm[(ty + 16 * a) * LB_LD + tx + 16 * b] -= acc[a][b];
+    }
+    __syncthreads();
+}
+
+template <int KB>
+__device__ __forceinline__ void leaf_block(float *Sm, float *Xm, float *Tm, float *rowbuf,
+                                           long long col_base, int tid) {
+    if (tid < 32) leaf_diag32(Sm, Xm, rowbuf, KB * LB, col_base, tid);
+    __syncthreads();
+    leaf_block_updates<KB>(Sm, Xm, Tm, tid);
+}
 
 __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, long long lda,
                                                                 float *U, long long ldu, int nb,
                                                                 long long col_base) {
     extern __shared__ __align__(16) float lsm[];
-    float *Sm = lsm;                                  // [128][129] Schur complement / panels
-    float *Xm = Sm + FACTOR_NB * LB_LD;               // [128][129] the inverse (upper)
-    float *Tm = Xm + FACTOR_NB * LB_LD;               // [32][97]   Ubar[k, >k] X[>k, >k]
-    float *xb = Tm + LB * LB_TLD;                     // [2][2][32] step exchange (u, row c)
-    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-
+    float *Sm = lsm;                                  // [128][132] Schur complement / panels
+    float *Xm = Sm + FACTOR_NB * LB_LD;               // [128][132] the inverse (upper)
+    float *Tm = Xm + FACTOR_NB * LB_LD;               // [32][100]  Ubar[k, >k] X[>k, >k]
+    float *rowbuf = Tm + LB * LB_TLD;                 // [2][32]    row c of step c
+    const int tid = threadIdx.x;
 #pragma unroll 4
     for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
         const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
@@ -379,159 +387,10 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
         Xm[i * LB_LD + j] = 0.f;
     }
     __syncthreads();
-
-#pragma unroll 1
-    for (int kb = FACTOR_NB / LB - 1; kb >= 0; --kb) {
-        const int r = kb * LB;
-        const int q = FACTOR_NB - r - LB;             // columns right of block k
-        // ---- A: the diagonal block -------------------------------------------------------
-        if (w == 0) {
-            const int i = lane;
-            float m[LB];
-#pragma unroll
-            for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
-#pragma unroll
-            for (int c = LB - 1; c >= 0; --c) {
-                float *ub = xb + (c & 1) * 2 * LB, *rb = ub + LB;
-                const float d = __shfl_sync(0xffffffffu, m[c], c);
-                const bool bad = !(d > 0.f) || !isfinite(d);
-                if (bad && i == 0) report(GPTQ_ERR_NOT_PD, col_base + r + c);
-                const float dd = bad ? 1.f : d;
-                float ip = rsqrtf(dd);
-                ip = ip * (1.5f - 0.5f * dd * ip * ip);  // one Newton step
-                const float u = i < c ? m[c] * ip : 0.f;
-                ub[i] = -u;
-                if (i == c) {
-#pragma unroll
-                    for (int j = c + 1; j < LB; ++j) rb[j] = -ip * m[j];
-                }
-                __syncwarp();
-                if (i == c) {
-                    m[c] = ip;
-#pragma unroll
-                    for (int j = c + 1; j < LB; ++j) m[j] = rb[j];
-                } else {
-#pragma unroll
-                    for (int j = 0; j < c; ++j) m[j] = fmaf(u, ub[j], m[j]);
-                    m[c] = u * ip;
-#pragma unroll
-                    for (int j = c + 1; j < LB; ++j) m[j] = fmaf(u, rb[j], m[j]);
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < LB; ++j) Xm[(r + i) * LB_LD + r + j] = j >= i ? m[j] : 0.f;
-        }
-        __syncthreads();
-        // ---- B (compute) and D1 ----------------------------------------------------------
-        float pb[12];
-        if (r > 0) {
-#pragma unroll
-            for (int t = 0; t < 12; ++t) pb[t] = 0.f;
-            const int c = lane;
-#pragma unroll 4
-            for (int mm = 0; mm < LB; ++mm) {
-                const float x = Xm[(r + c) * LB_LD + r + mm];
-#pragma unroll
-                for (int t = 0; t < 12; ++t)
-                    if (w + 8 * t < r) pb[t] = fmaf(Sm[(w + 8 * t) * LB_LD + r + mm], x, pb[t]);
-            }
-        }
-        if (q > 0) {
-            float acc[4][3];
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int h = 0; h < 3; ++h) acc[p][h] = 0.f;
-            for (int mm = r + LB; mm < FACTOR_NB; ++mm) {
-                float x[3], sv[4];
-#pragma unroll
-                for (int h = 0; h < 3; ++h) {
-                    const int jj = lane + 32 * h;
-                    x[h] = jj < q ? Xm[mm * LB_LD + r + LB + jj] : 0.f;
-                }
-#pragma unroll
-                for (int p = 0; p < 4; ++p) sv[p] = Sm[(r + w + 8 * p) * LB_LD + mm];
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-#pragma unroll
-                    for (int h = 0; h < 3; ++h) acc[p][h] = fmaf(sv[p], x[h], acc[p][h]);
-            }
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int h = 0; h < 3; ++h) {
-                    const int jj = lane + 32 * h;
-                    if (jj < q) Tm[(w + 8 * p) * LB_TLD + jj] = acc[p][h];
-                }
-        }
-        __syncthreads();
-        // ---- B (write) and D2 ------------------------------------------------------------
-        if (r > 0) {
-#pragma unroll
-            for (int t = 0; t < 12; ++t)
-                if (w + 8 * t < r) Sm[(w + 8 * t) * LB_LD + r + lane] = pb[t];
-        }
-        if (q > 0) {
-            float acc[4][3];
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int h = 0; h < 3; ++h) acc[p][h] = 0.f;
-#pragma unroll 4
-            for (int c2 = 0; c2 < LB; ++c2) {
-                float x[4], tv[3];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) x[p] = Xm[(r + w + 8 * p) * LB_LD + r + c2];
-#pragma unroll
-                for (int h = 0; h < 3; ++h) {
-                    const int jj = lane + 32 * h;
-                    tv[h] = jj < q ? Tm[c2 * LB_TLD + jj] : 0.f;
-                }
-#pragma unroll
-                for (int p = 0; p < 4; ++p)
-#pragma unroll
-                    for (int h = 0; h < 3; ++h) acc[p][h] = fmaf(x[p], tv[h], acc[p][h]);
-            }
-#pragma unroll
-            for (int p = 0; p < 4; ++p)
-#pragma unroll
-                for (int h = 0; h < 3; ++h) {
-                    const int jj = lane + 32 * h;
-                    if (jj < q) Xm[(r + w + 8 * p) * LB_LD + r + LB + jj] = -acc[p][h];
-                }
-        }
-        __syncthreads();
-        // ---- C: the Schur complement -----------------------------------------------------
-        if (r > 0) {
-            const int tx = tid & 15, ty = tid >> 4;
-            float acc[6][6];
-#pragma unroll
-            for (int a = 0; a < 6; ++a)
-#pragma unroll
-                for (int b = 0; b < 6; ++b) acc[a][b] = 0.f;
-#pragma unroll 2
-            for (int c = 0; c < LB; ++c) {
-                float pa[6], pbv[6];
-#pragma unroll
-                for (int a = 0; a < 6; ++a) {
-                    pa[a] = ty + 16 * a < r ? Sm[(ty + 16 * a) * LB_LD + r + c] : 0.f;
-                    pbv[a] = tx + 16 * a < r ? Sm[(tx + 16 * a) * LB_LD + r + c] : 0.f;
-                }
-#pragma unroll
-                for (int a = 0; a < 6; ++a)
-#pragma unroll
-                    for (int b = 0; b < 6; ++b) acc[a][b] = fmaf(pa[a], pbv[b], acc[a][b]);
-            }
-#pragma unroll
-            for (int a = 0; a < 6; ++a)
-#pragma unroll
-                for (int b = 0; b < 6; ++b) {
-                    const int i = ty + 16 * a, j = tx + 16 * b;
-                    if (i < r && j < r) Sm[i * LB_LD + j] -= acc[a][b];
-                }
-        }
-        __syncthreads();
-    }
+    leaf_block<3>(Sm, Xm, Tm, rowbuf, col_base, tid);
+    leaf_block<2>(Sm, Xm, Tm, rowbuf, col_base, tid);
+    leaf_block<1>(Sm, Xm, Tm, rowbuf, col_base, tid);
+    leaf_block<0>(Sm, Xm, Tm, rowbuf, col_base, tid);
 #pragma unroll 4
     for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
         const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
@@ -541,21 +400,12 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
 
 inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, int nb,
                        long long col_base, cudaStream_t s) {
-    // GPTQ_LEAF: 0 the barrier-synchronised leaf (diag_ul_inv_kernel), 1 (default) the
-    // warp-owner leaf, 2 the blocked leaf
-    static const long long leaf = tc::env_ll("GPTQ_LEAF", 1);
-    if (leaf == 0) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
-    if (leaf == 2) {
-        cudaFuncSetAttribute(leaf_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)LEAF_BLK_SMEM);
-        leaf_blk_kernel<<<1, LEAF_THREADS, LEAF_BLK_SMEM, s>>>(A, lda, U, ldu, nb, col_base);
-        return launch_status();
-    }
-    cudaFuncSetAttribute(leaf_ul_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)LEAF_SMEM);
-    // clock cycles a warp waits for a step before the kernel gives up with GPTQ_ERR_TIMEOUT
-    static const long long limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
-    leaf_ul_inv_kernel<<<1, LEAF_THREADS, LEAF_SMEM, s>>>(A, lda, U, ldu, nb, col_base, limit);
+    // GPTQ_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
+    static const bool blocked = tc::env_ll("GPTQ_LEAF", 1) != 0;
+    if (!blocked) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
+    cudaFuncSetAttribute(leaf_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)LEAF_BLK_SMEM);
+    leaf_blk_kernel<<<1, LEAF_THREADS, LEAF_BLK_SMEM, s>>>(A, lda, U, ldu, nb, col_base);
     return launch_status();
 }
 

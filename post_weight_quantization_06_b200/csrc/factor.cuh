@@ -183,8 +183,8 @@ __global__ void copy_damped_kernel(const float *H, long long ldh, float *A, long
 //      (S[c, j] = S[j, c] for j < c), so lane c's row is the only thing exchanged (one
 //      shared-memory row per step) and every lane applies m_j += a r_j with one scalar a
 //      (-u_i / sqrt(d) for rows above c, -1 - 1/sqrt(d) for row c itself, which turns its
-//      entries right of c into row c of the inverse, 0 below). Registers rotate by 4 every
-//      4 steps so the pivot's register index is static while the loop stays short;
+//      entries right of c into row c of the inverse, 0 below). Registers rotate by one per
+//      step so the pivot's register index is static and the loop body is one step;
 //   B  Ubar's panel Ubar[0:r, k] = S[0:r, k] X_kk^T, written over S[0:r, k];
 //   C  S[0:r, 0:r] -= Ubar[0:r, k] Ubar[0:r, k]^T;
 //   D  X[k, >k] = -X_kk (Ubar[k, >k] X[>k, >k]): the inverse's rows right of the diagonal.
@@ -197,56 +197,47 @@ constexpr int LEAF_THREADS = 256;
 constexpr size_t LEAF_BLK_SMEM =
     sizeof(float) * (2 * (size_t)FACTOR_NB * LB_LD + (size_t)LB * LB_TLD + 2 * LB);
 
-template <int R>
-__device__ __forceinline__ void rotate_right(float (&x)[LB]) {
-    float t[R];
-#pragma unroll
-    for (int k = 0; k < R; ++k) t[k] = x[LB - R + k];
-#pragma unroll
-    for (int k = LB - 1; k >= R; --k) x[k] = x[k - R];
-#pragma unroll
-    for (int k = 0; k < R; ++k) x[k] = t[k];
-}
-
-// A: X_kk of the 32 x 32 block of S at (r, r), written to X (warp 0 only).
+// A: X_kk of the 32 x 32 block of S at (r, r), written to X (warp 0 only). Before step c,
+// physical register p holds column (p - 31 + c) mod 32, so the pivot is always m[31]; the
+// rotation by one that keeps it there is folded into the update, and the loop body is one
+// step (a short body also keeps the first, cold pass through the code cheap).
 __device__ __forceinline__ void leaf_diag32(float *Sm, float *Xm, float *rowbuf, int r,
                                             long long col_base, int i) {
     float m[LB];
 #pragma unroll
     for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
-    // physical register p holds column (p - 31 + c0) mod 32 while steps c0 .. c0 - 3 run
 #pragma unroll 1
-    for (int c0 = LB - 1; c0 >= 0; c0 -= 4) {
+    for (int c = LB - 1; c >= 0; --c) {
+        float *rb = rowbuf + (c & 1) * LB;
+        if (i == c) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int c = c0 - u, P = LB - 1 - u;
-            float *rb = rowbuf + (u & 1) * LB;
-            if (i == c) {
-#pragma unroll
-                for (int p4 = 0; p4 < LB; p4 += 4)
-                    *reinterpret_cast<float4 *>(rb + p4) = make_float4(m[p4], m[p4 + 1], m[p4 + 2], m[p4 + 3]);
-            }
-            const float d = __shfl_sync(0xffffffffu, m[P], c);
-            const bool bad = !(d > 0.f) || !isfinite(d);
-            if (bad && i == 0) report(GPTQ_ERR_NOT_PD, col_base + r + c);
-            const float dd = bad ? 1.f : d;
-            float ip = rsqrtf(dd);
-            ip = ip * (1.5f - 0.5f * dd * ip * ip);  // one Newton step
-            const float uu = m[P] * ip;
-            const float a = i < c ? -uu * ip : (i == c ? -1.f - ip : 0.f);
-            __syncwarp();
-            float rv[LB];
-#pragma unroll
-            for (int p4 = 0; p4 < LB; p4 += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(rb + p4);
-                rv[p4] = t4.x; rv[p4 + 1] = t4.y; rv[p4 + 2] = t4.z; rv[p4 + 3] = t4.w;
-            }
-#pragma unroll
-            for (int p = 0; p < LB; ++p)
-                if (p != P) m[p] = fmaf(a, rv[p], m[p]);
-            m[P] = i < c ? uu * ip : ip;
+            for (int p4 = 0; p4 < LB; p4 += 4)
+                *reinterpret_cast<float4 *>(rb + p4) = make_float4(m[p4], m[p4 + 1], m[p4 + 2], m[p4 + 3]);
         }
-        rotate_right<4>(m);
+        const float d = __shfl_sync(0xffffffffu, m[LB - 1], c);
+        const bool bad = !(d > 0.f) || !isfinite(d);
+        if (bad && i == 0) report(GPTQ_ERR_NOT_PD, col_base + r + c);
+        const float dd = bad ? 1.f : d;
+        float ip = rsqrtf(dd);
+        ip = ip * (1.5f - 0.5f * dd * ip * ip);  // one Newton step
+        const float uu = m[LB - 1] * ip;
+        const float a = i < c ? -uu * ip : (i == c ? -1.f - ip : 0.f);
+        __syncwarp();
+        // new_p = m_p + a r_p (p < 31), new_31 = the restarted pivot entry; m_{p+1} <- new_p
+        const float piv = i < c ? uu * ip : ip;
+        float prev = piv;
+#pragma unroll
+        for (int p4 = 0; p4 < LB - 4; p4 += 4) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(rb + p4);
+            const float n0 = fmaf(a, t4.x, m[p4]), n1 = fmaf(a, t4.y, m[p4 + 1]);
+            const float n2 = fmaf(a, t4.z, m[p4 + 2]), n3 = fmaf(a, t4.w, m[p4 + 3]);
+            m[p4] = prev; m[p4 + 1] = n0; m[p4 + 2] = n1; m[p4 + 3] = n2;
+            prev = n3;
+        }
+        const float4 t4 = *reinterpret_cast<const float4 *>(rb + LB - 4);
+        const float n0 = fmaf(a, t4.x, m[LB - 4]), n1 = fmaf(a, t4.y, m[LB - 3]);
+        const float n2 = fmaf(a, t4.z, m[LB - 2]);
+        m[LB - 4] = prev; m[LB - 3] = n0; m[LB - 2] = n1; m[LB - 1] = n2;
     }
 #pragma unroll
     for (int j = 0; j < LB; ++j) Xm[(r + i) * LB_LD + r + j] = j >= i ? m[j] : 0.f;
@@ -377,13 +368,15 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
     float *Tm = Xm + FACTOR_NB * LB_LD;               // [32][100]  Ubar[k, >k] X[>k, >k]
     float *rowbuf = Tm + LB * LB_TLD;                 // [2][32]    row c of step c
     const int tid = threadIdx.x;
-#pragma unroll 4
+    // stage S symmetrically from A's upper triangle (coalesced rows, all loads in flight)
+#pragma unroll 16
     for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
         const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
-        float v;
-        if (i < nb && j < nb) v = j >= i ? A[(long long)i * lda + j] : A[(long long)j * lda + i];
-        else v = i == j ? 1.f : 0.f;
-        Sm[i * LB_LD + j] = v;
+        if (j >= i) {
+            const float v = (i < nb && j < nb) ? A[(long long)i * lda + j] : (i == j ? 1.f : 0.f);
+            Sm[i * LB_LD + j] = v;
+            Sm[j * LB_LD + i] = v;
+        }
         Xm[i * LB_LD + j] = 0.f;
     }
     __syncthreads();

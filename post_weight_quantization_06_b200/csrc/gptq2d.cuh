@@ -76,19 +76,9 @@ constexpr int UHS_PITCH = T2D + 4;
 // tile (up to W - 1 per direction)
 inline size_t gptq2d_sweep_smem(int band) { return sizeof(float) * T2D_TILE * (10 + 4 * (band - 1)); }
 
-// Physical register p of a rotated row holds slot (base + p) % 32; shifting the array down by
-// R after R steps keeps the slot of the current step at index 0 .. R-1.
-template <int R>
-__device__ __forceinline__ void rotate_down(float (&x)[T2D]) {
-    float t[R];
-#pragma unroll
-    for (int i = 0; i < R; ++i) t[i] = x[i];
-#pragma unroll
-    for (int i = 0; i < T2D - R; ++i) x[i] = x[i + R];
-#pragma unroll
-    for (int i = 0; i < R; ++i) x[T2D - R + i] = t[i];
-}
-
+// Physical register p of a rotated row holds slot (base + p) % 32; the rows are kept as pairs
+// of slots, and rotating the pair array down by R pairs after 2R steps keeps the slot of the
+// current step at index 0 .. 2R-1.
 template <int R>
 __device__ __forceinline__ void rotate_down2(float2 (&x)[T2D / 2]) {
     float2 t[R];

@@ -75,23 +75,32 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarps = blockDim.x >> 5;
     const int j0 = a.j0;
-    // U block load: eight independent global loads in flight per thread before the stores
-    for (int base = tid; base < B * B; base += 8 * blockDim.x) {
-        float v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int idx = base + u * blockDim.x;
-            v[u] = idx < B * B ? a.U[(long long)(j0 + idx / B) * a.ldu + j0 + idx % B] : 0.f;
+    // U block load: with 16-byte aligned rows all of it goes out at once as cp.async (the
+    // weight rows below load meanwhile); otherwise eight plain loads in flight per thread
+    const bool async_u = ((reinterpret_cast<uintptr_t>(a.U) | (uintptr_t)(a.ldu * 4)) & 15u) == 0;
+    if (async_u) {
+        for (int c = tid; c < B * B / 4; c += blockDim.x) {
+            const int row = c / (B / 4), q4 = (c % (B / 4)) * 4;
+            const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(Us + row * B + q4));
+            const float *src = a.U + (long long)(j0 + row) * a.ldu + j0 + q4;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
         }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    } else {
+        for (int base = tid; base < B * B; base += 8 * blockDim.x) {
+            float v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int idx = base + u * blockDim.x;
-            if (idx < B * B) Us[idx] = v[u];
+            for (int u = 0; u < 8; ++u) {
+                const int idx = base + u * blockDim.x;
+                v[u] = idx < B * B ? a.U[(long long)(j0 + idx / B) * a.ldu + j0 + idx % B] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int idx = base + u * blockDim.x;
+                if (idx < B * B) Us[idx] = v[u];
+            }
         }
     }
-    __syncthreads();
-    for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
-    __syncthreads();
 
     const int maxq = (1 << a.bits) - 1;
     const float fmaxq = (float)maxq;
@@ -113,6 +122,10 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
             cv[r][q] = 0;
         }
     }
+    if (async_u) asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+    __syncthreads();
+    for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
+    __syncthreads();
     const int gs = a.gs;
     const bool groups_in_panel = gs <= B;  // then B % gs == 0
     if (!groups_in_panel) {

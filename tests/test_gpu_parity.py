@@ -201,6 +201,32 @@ def test_quantize_stage_matches_oracle(g, m, n, bits, gs, B, wdt):
     assert np.all(np.abs(zeros.cpu().numpy() - zr) <= 0.5 + CODE_BAND)
 
 
+def test_quantize_with_unaligned_factor_rows_is_identical(g):
+    """U starting 4 bytes past a 16-byte boundary takes the column loop's plain-load path for
+    its U blocks; the result must equal the cp.async path's bit for bit."""
+    m, n, bits, gs, B = 48, 512, 4, 128, 128
+    X = _spd_from_data(n, 4 * n, 7)
+    Hd, _ = oracle.damp(oracle.hessian(X), 0.01)
+    U32 = torch.from_numpy(np.ascontiguousarray(oracle.inverse_cholesky_upper(Hd).astype(np.float32))).to(DEV)
+    buf = torch.empty(n * n + 1, device=DEV)
+    Umis = buf[1:].view(n, n)
+    Umis.copy_(U32)
+    assert Umis.data_ptr() % 16 == 4
+    W = torch.from_numpy(_rng(3).standard_normal((m, n)) * 0.02).float().to(DEV)
+    outs = []
+    for U in (U32, Umis):
+        codes = torch.empty(m, n * bits // 32, dtype=torch.int32, device=DEV)
+        scales = torch.empty(m, n // gs, device=DEV)
+        zeros = torch.empty(m, n // gs, dtype=torch.uint8, device=DEV)
+        loss = torch.empty(m, dtype=torch.float64, device=DEV)
+        g.gptq_quantize_layer(W, U, bits, gs, B, codes, scales, zeros, loss,
+                              g.workspace(g.GPTQ_OP_QUANTIZE, m, n, 0, B))
+        g.gptq_sync_status()
+        outs.append((codes, scales, zeros, loss))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
+
+
 def test_quantize_reports_nonfinite_weight(g):
     m, n = 8, 128
     W = torch.zeros(m, n, device=DEV)
@@ -325,6 +351,12 @@ def test_il_lowrank_quarter(g):
 def test_il_small_rank(g):
     L = datagen.lowrank(device=DEV, scale=0.125, r=8)
     _e2e_il(g, L)
+
+
+def test_il_odd_rank(g):
+    """r = 5: the augmented rows (n + r floats) are not 16-byte multiples, so every product and
+    the column loop take their unaligned paths."""
+    _e2e_il(g, datagen.lowrank(device=DEV, scale=0.125, r=5))
 
 
 def test_il_r0_equals_plain(g):

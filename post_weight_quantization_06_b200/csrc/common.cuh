@@ -70,6 +70,31 @@ inline int launch_status() {
     return e == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }
 
+// Programmatic dependent launch: a kernel launched with `pdl` may start while the previous
+// kernel of its stream is still running; it must call pdl_wait_prev() before touching what
+// that kernel writes. pdl_launch_next() lets the next such kernel start. Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline int launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                         cudaStream_t s, bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, args...);
+    const int st = launch_status();
+    return e == cudaSuccess ? st : GPTQ_ERR_CUDA;
+}
+
 #define GPTQ_CHECK_LAUNCH()                  \
     do {                                     \
         int _s = ::gptq::launch_status();    \

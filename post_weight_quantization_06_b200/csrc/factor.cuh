@@ -368,6 +368,7 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
     float *Tm = Xm + FACTOR_NB * LB_LD;               // [32][100]  Ubar[k, >k] X[>k, >k]
     float *rowbuf = Tm + LB * LB_TLD;                 // [2][32]    row c of step c
     const int tid = threadIdx.x;
+    pdl_wait_prev();
     // stage S symmetrically from A's upper triangle (coalesced rows, all loads in flight)
 #pragma unroll 16
     for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
@@ -384,6 +385,7 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
     leaf_block<2>(Sm, Xm, Tm, rowbuf, col_base, tid);
     leaf_block<1>(Sm, Xm, Tm, rowbuf, col_base, tid);
     leaf_block<0>(Sm, Xm, Tm, rowbuf, col_base, tid);
+    pdl_launch_next();
 #pragma unroll 4
     for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
         const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
@@ -391,15 +393,16 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
     }
 }
 
+// pdl: launch as a programmatic dependent of the stream's previous kernel.
 inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, int nb,
-                       long long col_base, cudaStream_t s) {
+                       long long col_base, cudaStream_t s, bool pdl = false) {
     // GPTQ_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
     static const bool blocked = tc::env_ll("GPTQ_LEAF", 1) != 0;
     if (!blocked) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
     cudaFuncSetAttribute(leaf_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)LEAF_BLK_SMEM);
-    leaf_blk_kernel<<<1, LEAF_THREADS, LEAF_BLK_SMEM, s>>>(A, lda, U, ldu, nb, col_base);
-    return launch_status();
+    return launch_kernel(leaf_blk_kernel, dim3(1), dim3(LEAF_THREADS), LEAF_BLK_SMEM, s, pdl, A,
+                         lda, U, ldu, nb, col_base);
 }
 
 // Streams of the blocked factor: the pivot chain (leaf, panel solve, look-ahead column) on a
@@ -474,10 +477,12 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
         const int r = k * FACTOR_NB, bk = std::min(FACTOR_NB, n - r);
         float *Xkk = U + (long long)r * ldu + r;
         float *Lt = A + (long long)r * lda;  // L_k^T: bk x r, strict lower block row k
-        if ((st = leaf_ul_inv(A + (long long)r * lda + r, lda, Xkk, ldu, bk, r, fs->chain))) break;
+        // the chain's leaf and panel product start while their predecessors finish
+        if ((st = leaf_ul_inv(A + (long long)r * lda + r, lda, Xkk, ldu, bk, r, fs->chain, true))) break;
         if (k > 0) {
             auto p = gemm_args<float, float>(bk, r, bk, Xkk, ldu, 0, A + r, lda, 1, Lt, lda, 1.f, 0.f);
             p.a_upper = 1;
+            p.pdl = 1;
             // the chain's products are small (K = 128, at most 47 output tiles of 128): the SIMT
             // kernel's 64-tiles start sooner and spread wider than the tensor-core pipeline
             if ((st = gemm_simt(p, fs->chain))) break;
@@ -488,6 +493,7 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
             cudaStreamWaitEvent(fs->chain, fs->bulk_done, 0);  // bulk update of block k+1
             auto p = gemm_args<float, float>(r, FACTOR_NB, bk, Lt, lda, 1, Lt + r1, lda, 0, A + r1,
                                              lda, -1.f, 1.f);
+            p.pdl = 1;
             if ((st = gemm_simt(p, fs->chain))) break;
             if (r1 > 0) {
                 cudaStreamWaitEvent(fs->bulk, fs->panel, 0);

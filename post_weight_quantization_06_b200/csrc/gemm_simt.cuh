@@ -26,6 +26,8 @@ struct GemmArgs {
     int b_lower;        // B(k,j) = 0 for k < j
     int max_ctas;       // > 0: at most this many persistent CTAs (tensor-core path only), so
                         // that kernels on other streams keep SMs
+    int pdl;            // SIMT path: launch as a programmatic dependent of the stream's previous
+                        // kernel (the launch overlaps that kernel's tail)
 };
 
 namespace simt {
@@ -41,6 +43,7 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
     constexpr int BM = BT, BN = BT, BK = 2048 / BT, TM = BT / 16, NH = TM / 4;
     const int i0 = blockIdx.y * BM, j0 = blockIdx.x * BN;
     if (p.c_upper && i0 >= j0 + BN) return;
+    pdl_wait_prev();
     __shared__ __align__(16) float As[BK][BM + 4];
     __shared__ __align__(16) float Bs[BK][BN + 4];
     const int tid = threadIdx.x;
@@ -120,6 +123,7 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
         }
         __syncthreads();
     }
+    pdl_launch_next();
     // epilogue: with beta != 0 every read of C is issued before the first write (one round
     // trip instead of one per element)
     if (p.beta != 0.f) {
@@ -159,12 +163,10 @@ inline int gemm_simt(const GemmArgs<TA, TB> &p, cudaStream_t s) {
     // fewer than ~one 128-tile wave: use 64 x 64 tiles for four times the CTAs
     if ((long long)ceil_div(p.M, 128) * ceil_div(p.N, 128) < 148) {
         dim3 grid(ceil_div(p.N, 64), ceil_div(p.M, 64));
-        gemm_simt_kernel<TA, TB, 64><<<grid, simt::NT, 0, s>>>(p);
-    } else {
-        dim3 grid(ceil_div(p.N, 128), ceil_div(p.M, 128));
-        gemm_simt_kernel<TA, TB, 128><<<grid, simt::NT, 0, s>>>(p);
+        return launch_kernel(gemm_simt_kernel<TA, TB, 64>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
     }
-    return launch_status();
+    dim3 grid(ceil_div(p.N, 128), ceil_div(p.M, 128));
+    return launch_kernel(gemm_simt_kernel<TA, TB, 128>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
 }
 
 template <typename TA, typename TB>
@@ -179,6 +181,7 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.alpha = alpha; p.beta = beta;
     p.c_upper = 0; p.a_upper = 0; p.b_upper = 0; p.a_lower = 0; p.b_lower = 0;
     p.max_ctas = 0;
+    p.pdl = 0;
     return p;
 }
 

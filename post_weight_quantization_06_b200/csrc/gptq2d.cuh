@@ -46,11 +46,9 @@ struct Gptq2dArgs {
     int m, n, MT, NT;
 };
 
-// Programmatic dependent launch: every kernel of the wavefront lets the next one start at
-// once (its independent prologue overlaps this kernel) and waits for the previous kernel's
-// completion before it touches anything that kernel wrote.
-__device__ __forceinline__ void pdl_launch_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-__device__ __forceinline__ void pdl_wait_prev() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Programmatic dependent launch (common.cuh): every kernel of the wavefront lets the next one
+// start at once (its independent prologue overlaps this kernel) and waits for the previous
+// kernel's completion before it touches anything that kernel wrote.
 
 __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
     const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
@@ -502,21 +500,7 @@ __global__ void gptq2d_pad_identity_kernel(float *U, long long d0, long long dp)
 template <typename... KArgs, typename... Args>
 inline int launch_pdl(void (*kernel)(KArgs...), dim3 grid, int threads, size_t smem,
                       cudaStream_t s, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(threads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) {
-        launch_status();
-        return GPTQ_ERR_CUDA;
-    }
-    return launch_status();
+    return launch_kernel(kernel, grid, dim3(threads), smem, s, true, args...);
 }
 
 // Side stream on which U_G is factored while U_H is factored on the caller's stream (one per

@@ -127,7 +127,8 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
     __syncthreads();
     const int gs = a.gs;
-    const bool groups_in_panel = gs <= B;  // then B % gs == 0
+    const bool groups_in_panel = gs <= B;  // then B % gs == 0, so gs is a power of two
+    const int gmask = groups_in_panel ? gs - 1 : 0;
     if (!groups_in_panel) {
         const int g = j0 / gs;
         if (j0 % gs == 0) {
@@ -168,7 +169,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
 #pragma unroll 2
         for (int o = 0; o < 32; ++o) {
             const int t = 32 * q + o;
-            if (groups_in_panel && (t % gs) == 0) {
+            if (groups_in_panel && (t & gmask) == 0) {
                 const int g = (j0 + t) / gs;
 #pragma unroll
                 for (int r = 0; r < ROWS; ++r) {

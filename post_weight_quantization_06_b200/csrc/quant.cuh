@@ -106,7 +106,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     const float fmaxq = (float)maxq;
     const int row0 = (blockIdx.x * nwarps + warp) * ROWS;
     float w[ROWS][NSLOT], ev[ROWS][NSLOT];
-    int cv[ROWS][NSLOT];
+    float cv[ROWS][NSLOT];   // codes kept as floats until the panel is done
     float s[ROWS], is[ROWS], z[ROWS], lacc[ROWS];
     bool rv[ROWS];
 #pragma unroll
@@ -119,7 +119,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
         for (int q = 0; q < NSLOT; ++q) {
             w[r][q] = rv[r] ? a.Wc[(long long)row * a.ldw + j0 + 32 * q + lane] : 0.f;
             ev[r][q] = 0.f;
-            cv[r][q] = 0;
+            cv[r][q] = 0.f;
         }
     }
     if (async_u) asm volatile("cp.async.wait_group 0;\n" ::: "memory");
@@ -166,7 +166,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
 
 #pragma unroll
     for (int q = 0; q < NSLOT; ++q) {
-#pragma unroll 2
+#pragma unroll 4
         for (int o = 0; o < 32; ++o) {
             const int t = 32 * q + o;
             if (groups_in_panel && (t & gmask) == 0) {
@@ -202,7 +202,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
                 const float e = (wt - wq) * ut;
                 lacc[r] = fmaf(e, e, lacc[r]);
                 if (lane == o) {
-                    cv[r][q] = (int)c;
+                    cv[r][q] = c;
                     ev[r][q] = e;
                 }
 #pragma unroll
@@ -222,7 +222,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
 #pragma unroll
         for (int q = 0; q < NSLOT; ++q) {
             if (rv[r]) a.err[(long long)row * a.lde + 32 * q + lane] = ev[r][q];
-            cb[r * B + 32 * q + lane] = (uint8_t)cv[r][q];
+            cb[r * B + 32 * q + lane] = (uint8_t)(int)cv[r][q];
         }
         if (a.loss && lane == 0 && rv[r]) {
             if (j0 == 0) a.loss[row] = (double)lacc[r];

@@ -107,13 +107,12 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     const int row0 = (blockIdx.x * nwarps + warp) * ROWS;
     float w[ROWS][NSLOT], ev[ROWS][NSLOT];
     float cv[ROWS][NSLOT];   // codes kept as floats until the panel is done
-    float s[ROWS], is[ROWS], z[ROWS], lacc[ROWS];
+    float s[ROWS], is[ROWS], z[ROWS];
     bool rv[ROWS];
 #pragma unroll
     for (int r = 0; r < ROWS; ++r) {
         const int row = row0 + r;
         rv[r] = row < a.m;
-        lacc[r] = 0.f;
         s[r] = 1.f; is[r] = 1.f; z[r] = 0.f;
 #pragma unroll
         for (int q = 0; q < NSLOT; ++q) {
@@ -200,7 +199,6 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
                 const float c = fminf(fmaxf(rintf(v), 0.f), fmaxq);
                 const float wq = s[r] * (c - z[r]);
                 const float e = (wt - wq) * ut;
-                lacc[r] = fmaf(e, e, lacc[r]);
                 if (lane == o) {
                     cv[r][q] = c;
                     ev[r][q] = e;
@@ -224,9 +222,16 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
             if (rv[r]) a.err[(long long)row * a.lde + 32 * q + lane] = ev[r][q];
             cb[r * B + 32 * q + lane] = (uint8_t)(int)cv[r][q];
         }
-        if (a.loss && lane == 0 && rv[r]) {
-            if (j0 == 0) a.loss[row] = (double)lacc[r];
-            else a.loss[row] += (double)lacc[r];
+        if (a.loss) {
+            // the panel's share of the loss: each lane's own columns, then the warp's sum
+            double l = 0.0;
+#pragma unroll
+            for (int q = 0; q < NSLOT; ++q) l += (double)ev[r][q] * (double)ev[r][q];
+            l = warp_sum_d(l);
+            if (lane == 0 && rv[r]) {
+                if (j0 == 0) a.loss[row] = l;
+                else a.loss[row] += l;
+            }
         }
     }
     __syncwarp();

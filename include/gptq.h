@@ -11,6 +11,7 @@
  *   gptq_il_refine            OLrC + Bid-Up refinement rounds on a quantized layer: new L, R, codes
  *   gptq_quantize_lowrank     L and R stored at low precision (4-bit L, 8-bit R) on min-max grids
  *   gptq_2d_round             two-sided adaptive rounding of a real matrix to integers (GPTQ-2D)
+ *   gptq_set_flags            synchronous status returns and debug synchronisation (see below)
  *
  * Conventions shared by every entry point
  *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);
@@ -68,6 +69,25 @@ typedef enum {
     GPTQ_OP_IL_REFINE = 4,
     GPTQ_OP_2D_ROUND = 5
 } gptq_op;
+
+/* Process-wide behaviour flags (gptq_set_flags; default 0):
+ *   GPTQ_FLAG_SYNC_STATUS   every compute entry point synchronises its stream after enqueueing
+ *                           and returns the device status word (read and cleared, as
+ *                           gptq_sync_status does), so device-found errors are returned by the
+ *                           call that caused them.
+ *   GPTQ_FLAG_DEBUG_CHECKS  as SYNC_STATUS, after a device-wide synchronise that also surfaces
+ *                           errors of the library's side streams (GPTQ_ERR_CUDA).
+ *   GPTQ_FLAG_IL_FP64       accepted for compatibility: the intrinsic-LoRA path always forms its
+ *                           cancelling products (Gram matrices, Schur complement) with fp64
+ *                           accumulation. */
+typedef enum {
+    GPTQ_FLAG_SYNC_STATUS = 1u,
+    GPTQ_FLAG_DEBUG_CHECKS = 2u,
+    GPTQ_FLAG_IL_FP64 = 4u
+} gptq_flag;
+
+GPTQ_API void gptq_set_flags(unsigned flags);
+GPTQ_API unsigned gptq_get_flags(void);
 
 /* Bytes of device workspace the entry point `op` needs for these sizes (0 if none).
  * m, n: layer shape; r: intrinsic-LoRA rank (IL only, else 0); block_size: B.

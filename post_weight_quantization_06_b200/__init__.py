@@ -20,11 +20,12 @@ GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
 GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND = 4, 5
+GPTQ_FLAG_SYNC_STATUS, GPTQ_FLAG_DEBUG_CHECKS, GPTQ_FLAG_IL_FP64 = 1, 2, 4
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
             "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-            "gptq_quantize_lowrank", "gptq_2d_round")
+            "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags")
 
 
 class GptqError(RuntimeError):
@@ -58,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "gptq_quantize_lowrank": (c_int, [c_p, c_p, c_i64, c_i64, c_int, c_int, c_int, c_int,
                                           c_p, c_p, c_p, c_p, c_p, c_p, c_p]),
         "gptq_2d_round": (c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "gptq_set_flags": (None, [ctypes.c_uint]),
+        "gptq_get_flags": (ctypes.c_uint, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -111,6 +114,14 @@ def workspace(op: int, m: int, n: int, r: int = 0, block_size: int = 128, device
     """A caller-owned workspace tensor (uint8, 256-byte aligned by the caching allocator)."""
     nbytes = gptq_workspace_size(op, m, n, r, block_size)
     return torch.empty(max(nbytes, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def gptq_set_flags(flags: int) -> None:
+    _lib.gptq_set_flags(int(flags))
+
+
+def gptq_get_flags() -> int:
+    return int(_lib.gptq_get_flags())
 
 
 def gptq_launch_count() -> int:

@@ -1,5 +1,6 @@
 // libgptq: C ABI of the GPTQ / GPTQ-intrinsic-LoRA layer pass for sm_100a.
 // One translation unit: the kernels live in the included .cuh files.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -273,7 +274,22 @@ GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info) {
     return st.code;
 }
 
-GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64_t k, int64_t n,
+static std::atomic<unsigned> g_flags{0};
+
+GPTQ_API void gptq_set_flags(unsigned flags) { g_flags.store(flags); }
+GPTQ_API unsigned gptq_get_flags(void) { return g_flags.load(); }
+
+// Applied to the status of every compute entry point once its work is enqueued.
+static int finish_call(int st, gptq_stream_t stream) {
+    const unsigned f = g_flags.load();
+    if (st != GPTQ_OK || !(f & (GPTQ_FLAG_SYNC_STATUS | GPTQ_FLAG_DEBUG_CHECKS))) return st;
+    if ((f & GPTQ_FLAG_DEBUG_CHECKS) &&
+        (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess))
+        return GPTQ_ERR_CUDA;
+    return gptq_sync_status(stream, nullptr);
+}
+
+static int gptq_hessian_accumulate_body(float *H, const void *X, int x_dtype, int64_t k, int64_t n,
                                      gptq_stream_t stream) {
     if (!H || !X || k < 0 || n < 1 || n > 65536) return GPTQ_ERR_ARG;
     if (x_dtype != GPTQ_BF16 && x_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
@@ -293,7 +309,12 @@ GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64
     return hessian_simt(H, static_cast<const float *>(X), k, (int)n, s);
 }
 
-GPTQ_API int gptq_prepare_hinv(const float *H, int64_t n, float lambda_rel, float *U,
+GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64_t k, int64_t n,
+                                     gptq_stream_t stream) {
+    return finish_call(gptq_hessian_accumulate_body(H, X, x_dtype, k, n, stream), stream);
+}
+
+static int gptq_prepare_hinv_body(const float *H, int64_t n, float lambda_rel, float *U,
                                float *lambda_out, void *workspace, size_t ws_bytes,
                                gptq_stream_t stream) {
     if (!H || !U || !lambda_out || n < 1 || n > 65536) return GPTQ_ERR_ARG;
@@ -306,7 +327,15 @@ GPTQ_API int gptq_prepare_hinv(const float *H, int64_t n, float lambda_rel, floa
                              reinterpret_cast<cudaStream_t>(stream));
 }
 
-GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
+GPTQ_API int gptq_prepare_hinv(const float *H, int64_t n, float lambda_rel, float *U,
+                               float *lambda_out, void *workspace, size_t ws_bytes,
+                               gptq_stream_t stream) {
+    const int st = gptq_prepare_hinv_body(H, n, lambda_rel, U, lambda_out, workspace, ws_bytes,
+        stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_quantize_layer_body(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
                                  int bits, int group_size, int block_size, uint32_t *codes,
                                  float *scales, uint8_t *zeros, double *loss_out,
                                  void *workspace, size_t ws_bytes, gptq_stream_t stream) {
@@ -323,7 +352,16 @@ GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t 
                        codes, scales, zeros, loss_out, w.Err, s);
 }
 
-GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
+GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
+                                 int bits, int group_size, int block_size, uint32_t *codes,
+                                 float *scales, uint8_t *zeros, double *loss_out,
+                                 void *workspace, size_t ws_bytes, gptq_stream_t stream) {
+    const int st = gptq_quantize_layer_body(W, w_dtype, m, n, U, bits, group_size, block_size,
+        codes, scales, zeros, loss_out, workspace, ws_bytes, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_quantize_layer_noalloc_body(const void *W, int w_dtype, int64_t m, int64_t n,
                                          const float *U, int bits, int group_size,
                                          int block_size, uint32_t *codes, float *scales,
                                          uint8_t *zeros, double *loss_out,
@@ -345,7 +383,17 @@ GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, 
                        codes, scales, zeros, loss_out, w.Err, s);
 }
 
-GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n,
+GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
+                                         const float *U, int bits, int group_size,
+                                         int block_size, uint32_t *codes, float *scales,
+                                         uint8_t *zeros, double *loss_out,
+                                         gptq_stream_t stream) {
+    const int st = gptq_quantize_layer_noalloc_body(W, w_dtype, m, n, U, bits, group_size,
+        block_size, codes, scales, zeros, loss_out, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_il_quantize_layer_body(const void *W, int w_dtype, int64_t m, int64_t n,
                                     const float *H, int r, int bits, int group_size,
                                     float lambda_rel, int block_size, uint32_t *codes,
                                     float *scales, uint8_t *zeros, float *L, float *R,
@@ -382,7 +430,19 @@ GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64
     return GPTQ_OK;
 }
 
-GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
+GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n,
+                                    const float *H, int r, int bits, int group_size,
+                                    float lambda_rel, int block_size, uint32_t *codes,
+                                    float *scales, uint8_t *zeros, float *L, float *R,
+                                    float *lambda_out, double *loss_out, void *workspace,
+                                    size_t ws_bytes, gptq_stream_t stream) {
+    const int st = gptq_il_quantize_layer_body(W, w_dtype, m, n, H, r, bits, group_size,
+        lambda_rel, block_size, codes, scales, zeros, L, R, lambda_out, loss_out, workspace,
+        ws_bytes, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_il_refine_body(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
                             int r, int bits, int group_size, int iters, uint32_t *codes,
                             const float *scales, const uint8_t *zeros, float *L, float *R,
                             double *loss_hist, void *workspace, size_t ws_bytes,
@@ -415,7 +475,17 @@ GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, co
     return launch_status();
 }
 
-GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, int64_t m, int r,
+GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
+                            int r, int bits, int group_size, int iters, uint32_t *codes,
+                            const float *scales, const uint8_t *zeros, float *L, float *R,
+                            double *loss_hist, void *workspace, size_t ws_bytes,
+                            gptq_stream_t stream) {
+    const int st = gptq_il_refine_body(W, w_dtype, m, n, H, r, bits, group_size, iters, codes,
+        scales, zeros, L, R, loss_hist, workspace, ws_bytes, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_quantize_lowrank_body(const float *L, const float *R, int64_t n, int64_t m, int r,
                                    int bits_L, int group_size_L, int bits_R, uint32_t *codes_L,
                                    float *scales_L, uint8_t *zeros_L, uint32_t *codes_R,
                                    float *scales_R, uint8_t *zeros_R, gptq_stream_t stream) {
@@ -437,7 +507,16 @@ GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, in
     return launch_status();
 }
 
-GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G, const float *H,
+GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, int64_t m, int r,
+                                   int bits_L, int group_size_L, int bits_R, uint32_t *codes_L,
+                                   float *scales_L, uint8_t *zeros_L, uint32_t *codes_R,
+                                   float *scales_R, uint8_t *zeros_R, gptq_stream_t stream) {
+    const int st = gptq_quantize_lowrank_body(L, R, n, m, r, bits_L, group_size_L, bits_R,
+        codes_L, scales_L, zeros_L, codes_R, scales_R, zeros_R, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_2d_round_body(const float *X, int64_t m, int64_t n, const float *G, const float *H,
                            int32_t *Z, float *err, void *workspace, size_t ws_bytes,
                            gptq_stream_t stream) {
     if (m < 0 || n < 0 || m > 65536 || n > 65536) return GPTQ_ERR_ARG;
@@ -478,6 +557,13 @@ GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G,
     a.Z = Z; a.err = err; a.Mp = w.Mp; a.Np = w.Np; a.m = (int)m; a.n = (int)n;
     a.MT = (int)(w.Mp / T2D); a.NT = (int)(w.Np / T2D);
     return gptq2d_sweep(a, s);
+}
+
+GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G, const float *H,
+                           int32_t *Z, float *err, void *workspace, size_t ws_bytes,
+                           gptq_stream_t stream) {
+    const int st = gptq_2d_round_body(X, m, n, G, H, Z, err, workspace, ws_bytes, stream);
+    return finish_call(st, stream);
 }
 
 }  // extern "C"

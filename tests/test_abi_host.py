@@ -21,7 +21,7 @@ def test_header_declares_the_boundary():
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
         "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-        "gptq_quantize_lowrank", "gptq_2d_round"])
+        "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -190,3 +190,16 @@ def test_2d_round_checks_the_workspace_and_accepts_empty_input():
     # nothing to round: returns at once, touching no pointer
     assert lib.gptq_2d_round(NULL, 0, 70, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
     assert lib.gptq_2d_round(NULL, 40, 0, NULL, NULL, NULL, NULL, NULL, 0, NULL) == 0
+
+
+def test_flags_round_trip_and_host_errors_stay_synchronous():
+    import post_weight_quantization_06_b200 as g
+    try:
+        g.gptq_set_flags(g.GPTQ_FLAG_SYNC_STATUS | g.GPTQ_FLAG_IL_FP64)
+        assert g.gptq_get_flags() == g.GPTQ_FLAG_SYNC_STATUS | g.GPTQ_FLAG_IL_FP64
+        # argument errors are returned before anything is enqueued or synchronised
+        assert _lib().gptq_hessian_accumulate(NULL, P, 0, 10, 64, NULL) == -1
+        assert _lib().gptq_2d_round(P, -1, 5, P, P, P, NULL, NULL, 0, NULL) == -1
+    finally:
+        g.gptq_set_flags(0)
+    assert g.gptq_get_flags() == 0

@@ -3,6 +3,8 @@
 Stage tests feed each entry point the oracle's own inputs (H, U) so that one kernel family
 is judged at a time; end-to-end tests run the whole pass from X and W.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -144,6 +146,33 @@ def test_prepare_hinv_reports_non_positive_pivot(g):
     st, info = g.gptq_sync_status(raise_on_error=False)
     assert st == g.GPTQ_ERR_NOT_PD and info == 150
     assert g.gptq_sync_status() == (0, 0)   # cleared
+
+
+def test_sync_status_flag_returns_device_errors_from_the_call(g):
+    """GPTQ_FLAG_SYNC_STATUS: the failing call itself returns GPTQ_ERR_NOT_PD; a clean call
+    returns GPTQ_OK; with the flag cleared the error waits for gptq_sync_status again."""
+    n = 200
+    h = np.eye(n, dtype=np.float32)
+    h[150, 150] = -1.0
+    bad, good = torch.from_numpy(h).to(DEV), torch.eye(n, device=DEV)
+    U = torch.empty(n, n, device=DEV)
+    lam_t = torch.empty(1, device=DEV)
+    ws = g.workspace(g.GPTQ_OP_PREPARE_HINV, 0, n)
+    lib = g._lib
+    args = lambda H: (ctypes.c_void_p(H.data_ptr()), n, ctypes.c_float(0.0),
+                      ctypes.c_void_p(U.data_ptr()), ctypes.c_void_p(lam_t.data_ptr()),
+                      ctypes.c_void_p(ws.data_ptr()), ws.numel(), g._stream())
+    try:
+        g.gptq_set_flags(g.GPTQ_FLAG_SYNC_STATUS)
+        assert lib.gptq_prepare_hinv(*args(bad)) == g.GPTQ_ERR_NOT_PD
+        assert lib.gptq_prepare_hinv(*args(good)) == g.GPTQ_OK
+        g.gptq_set_flags(g.GPTQ_FLAG_DEBUG_CHECKS)
+        assert lib.gptq_prepare_hinv(*args(bad)) == g.GPTQ_ERR_NOT_PD
+    finally:
+        g.gptq_set_flags(0)
+    assert lib.gptq_prepare_hinv(*args(bad)) == g.GPTQ_OK
+    st, info = g.gptq_sync_status(raise_on_error=False)
+    assert st == g.GPTQ_ERR_NOT_PD and info == 150
 
 
 def test_prepare_hinv_reports_nonfinite_diagonal(g):

@@ -325,12 +325,31 @@ def run_refine(g, layer, lp, rounds):
     torch.cuda.synchronize(dev)
     h = hist.cpu().tolist()
     changed = int((codes != start).sum().item())   # packed words that differ
-    return {"rounds": rounds, "ms": e0.elapsed_time(e1), "ms_per_round": e0.elapsed_time(e1) / rounds,
+    ms_round = e0.elapsed_time(e1) / rounds
+    # product work of one round: g = D H (2 m n^2) and the Bid-Up lazy updates (about
+    # 2 m n^2); with r > 0 also E H and (E H) E^T for OLrC (2 m n^2 + 2 m^2 n)
+    flops = 4.0 * m * n * n + (2.0 * m * n * n + 2.0 * m * m * n if r else 0.0)
+    tf32x3 = tensor_peak_tflops() * TF32_PER_BF16 / 3.0
+    achieved = flops / (ms_round * 1e-3) / 1e12
+    return {"rounds": rounds, "ms": e0.elapsed_time(e1), "ms_per_round": ms_round,
+            "roofline": {"bound": "tensor", "kernel": "refinement round (tf32x3 products)",
+                         "achieved": achieved, "peak": tf32x3, "unit": "TFLOP/s",
+                         "frac": achieved / tf32x3,
+                         "peak_source": "measured bf16 sustained x nominal tf32/bf16 ratio / 3 passes"},
             "loss_after_first_olrc": h[0], "loss_final": h[-1],
             "loss_drop": (h[0] - h[-1]) / h[0] if h[0] else 0.0, "code_words_changed": changed}
 
 
 SIMT_FP32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # SMs x FP32 lanes x FMA x max SM clock
+TF32_PER_BF16 = 1.1 / 2.25                          # nominal dense tf32 : bf16 throughput
+
+
+def tensor_peak_tflops() -> float:
+    """Measured sustained bf16 tensor throughput (MEASURED_PEAKS.json), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["bf16_tflops_sustained"])
+    return 1400.0
 
 
 def run_gptq2d(g, dev, steps):

@@ -198,6 +198,10 @@ SWEEP_CASES = [
     (50, 256, 3, 64, 64, torch.float32),
     (33, 256, 4, 16, 32, torch.float32),
     (17, 128, 8, 128, 128, torch.float32),
+    # odd widths: codes straddle 32-bit words
+    (48, 256, 5, 64, 64, torch.float32),
+    (40, 512, 6, 128, 128, torch.bfloat16),
+    (36, 256, 7, 32, 32, torch.float32),
     # several 1024-column outer blocks of the two-level lazy update
     (64, 2560, 3, 128, 128, torch.bfloat16),
     (40, 2048, 4, 0, 128, torch.float32),

@@ -201,11 +201,8 @@ constexpr size_t LEAF_BLK_SMEM =
 // physical register p holds column (p - 31 + c) mod 32, so the pivot is always m[31]; the
 // rotation by one that keeps it there is folded into the update, and the loop body is one
 // step (a short body also keeps the first, cold pass through the code cheap).
-__device__ __forceinline__ void leaf_diag32(float *Sm, float *Xm, float *rowbuf, int r,
-                                            long long col_base, int i) {
-    float m[LB];
-#pragma unroll
-    for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
+__device__ __forceinline__ void leaf_diag32_regs(float (&m)[LB], float *Xm, float *rowbuf, int r,
+                                                 long long col_base, int i) {
 #pragma unroll 1
     for (int c = LB - 1; c >= 0; --c) {
         float *rb = rowbuf + (c & 1) * LB;
@@ -241,6 +238,14 @@ __device__ __forceinline__ void leaf_diag32(float *Sm, float *Xm, float *rowbuf,
     }
 #pragma unroll
     for (int j = 0; j < LB; ++j) Xm[(r + i) * LB_LD + r + j] = j >= i ? m[j] : 0.f;
+}
+
+__device__ __forceinline__ void leaf_diag32(float *Sm, float *Xm, float *rowbuf, int r,
+                                            long long col_base, int i) {
+    float m[LB];
+#pragma unroll
+    for (int j = 0; j < LB; ++j) m[j] = Sm[(r + i) * LB_LD + r + j];
+    leaf_diag32_regs(m, Xm, rowbuf, r, col_base, i);
 }
 
 // B, C, D of block KB (r = 32 KB rows above it, q = 96 - r columns right of it), 8 warps.
@@ -369,19 +374,37 @@ __global__ __launch_bounds__(LEAF_THREADS) void leaf_blk_kernel(const float *A, 
     float *rowbuf = Tm + LB * LB_TLD;                 // [2][32]    row c of step c
     const int tid = threadIdx.x;
     pdl_wait_prev();
-    // stage S symmetrically from A's upper triangle (coalesced rows, all loads in flight)
-#pragma unroll 16
-    for (int idx = tid; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS) {
-        const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
-        if (j >= i) {
-            const float v = (i < nb && j < nb) ? A[(long long)i * lda + j] : (i == j ? 1.f : 0.f);
-            Sm[i * LB_LD + j] = v;
-            Sm[j * LB_LD + i] = v;
+    constexpr int R3 = FACTOR_NB - LB;                // first column of the last 32-block
+    if (tid < 32) {
+        // warp 0 takes the last diagonal block straight from A and factors it while the other
+        // warps stage the rest (its first, instruction-cache-cold pass overlaps the staging)
+        float m[LB];
+        const int i = R3 + tid;
+#pragma unroll
+        for (int jj = 0; jj < LB; ++jj) {
+            const int j = R3 + jj;
+            float v;
+            if (i < nb && j < nb) v = j >= i ? A[(long long)i * lda + j] : A[(long long)j * lda + i];
+            else v = i == j ? 1.f : 0.f;
+            m[jj] = v;
         }
-        Xm[i * LB_LD + j] = 0.f;
+        leaf_diag32_regs(m, Xm, rowbuf, R3, col_base, tid);
+    } else {
+        // stage S symmetrically from A's upper triangle (coalesced rows); X starts at zero
+        // except the block warp 0 writes
+#pragma unroll 8
+        for (int idx = tid - 32; idx < FACTOR_NB * FACTOR_NB; idx += LEAF_THREADS - 32) {
+            const int i = idx >> 7, j = idx & (FACTOR_NB - 1);
+            if (j >= i) {
+                const float v = (i < nb && j < nb) ? A[(long long)i * lda + j] : (i == j ? 1.f : 0.f);
+                Sm[i * LB_LD + j] = v;
+                Sm[j * LB_LD + i] = v;
+            }
+            if (i < R3 || j < R3) Xm[i * LB_LD + j] = 0.f;
+        }
     }
     __syncthreads();
-    leaf_block<3>(Sm, Xm, Tm, rowbuf, col_base, tid);
+    leaf_block_updates<3>(Sm, Xm, Tm, tid);
     leaf_block<2>(Sm, Xm, Tm, rowbuf, col_base, tid);
     leaf_block<1>(Sm, Xm, Tm, rowbuf, col_base, tid);
     leaf_block<0>(Sm, Xm, Tm, rowbuf, col_base, tid);

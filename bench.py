@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=20.0)
     ap.add_argument("--refine-rounds", type=int, default=2,
                     help="OLrC + Bid-Up rounds timed after the pass (reported apart, 0: none)")
+    ap.add_argument("--no-gemm-times", action="store_true",
+                    help="skip the extra pass that times the fp32 GEMM launches per stage")
     ap.add_argument("--no-gptq2d", action="store_true",
                     help="skip the two-sided rounding (GPTQ-2D) timing reported under 'gptq2d'")
     ap.add_argument("--only-gptq2d", action="store_true",
@@ -352,6 +354,46 @@ def tensor_peak_tflops() -> float:
     return 1400.0
 
 
+def hbm_peak_gbs() -> float:
+    """Measured copy bandwidth (MEASURED_PEAKS.json), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        return float(json.load(open(path))["hbm_gbs"])
+    return 6650.0
+
+
+def run_gemm_times(g, lp):
+    """One more layer pass, outside the timed region, with GPTQ_FLAG_KERNEL_TIMES: the device
+    time and algorithmic work of the fp32 GEMM launches per stage (the factor's trailing and
+    inverse updates, the sweep's lazy updates) and path (tf32x3 tensor core, SIMT). A launch's
+    time runs from its start event to its stop event on its stream, so a factor update that
+    waits for SMs held by the chain counts the wait; the roofline time of a class is the larger
+    of its flops at the path's peak and its bytes at the measured HBM bandwidth."""
+    g.kernel_times()
+    g.gptq_set_flags(g.GPTQ_FLAG_KERNEL_TIMES)
+    try:
+        lp.step()
+        torch.cuda.synchronize()
+    finally:
+        g.gptq_set_flags(0)
+    kt = g.kernel_times()
+    tf32x3 = tensor_peak_tflops() * TF32_PER_BF16 / 3.0
+    hbm = hbm_peak_gbs()
+    out = {"peak_tc": tf32x3, "peak_simt": SIMT_FP32_TFLOPS, "hbm_gbs": hbm,
+           "peak_source": "tc: measured bf16 sustained x nominal tf32/bf16 ratio / 3 passes; "
+                          "simt: derived 148 SMs x 128 lanes x 2 x 1.965 GHz; hbm: measured copy"}
+    for (stage, path), v in sorted(kt.items()):
+        sec = v["ms"] * 1e-3
+        peak = tf32x3 if path == "tc" else SIMT_FP32_TFLOPS
+        t_roof = max(v["flops"] / (peak * 1e12), v["bytes"] / (hbm * 1e9))
+        out[f"{stage}_{path}"] = {
+            "launches": v["launches"], "ms": v["ms"], "gflop": v["flops"] / 1e9,
+            "gbytes": v["bytes"] / 1e9, "tflops": v["flops"] / sec / 1e12,
+            "frac_of_peak": v["flops"] / sec / 1e12 / peak, "roofline_ms": t_roof * 1e3,
+            "frac_of_roofline": t_roof / sec}
+    return out
+
+
 def run_gptq2d(g, dev, steps):
     """Two-sided rounding (gptq_2d_round) of X 2048 x 6144 under G 2048^2, H 6144^2: the whole
     call (both factorizations and the wavefront), and each factorization alone through
@@ -515,6 +557,8 @@ def bench_ours(args):
         peak, peak_src = 1400.0, "fallback (bf16 sustained)"
     h_tflops = hessian_flops(layer) / (stage[0] * 1e-3) / 1e12
 
+    gemm = run_gemm_times(g, lp) if not args.no_gemm_times else None
+
     refine = run_refine(g, layer, lp, args.refine_rounds) if args.refine_rounds > 0 else None
 
     two_d = run_gptq2d(g, dev, args.steps) if not args.no_gptq2d else None
@@ -556,6 +600,8 @@ def bench_ours(args):
         }
         if e2e:
             out["e2e"] = e2e
+        if gemm:
+            out["gemm"] = gemm
         if refine:
             out["refine"] = refine
         if two_d:

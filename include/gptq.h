@@ -79,11 +79,13 @@ typedef enum {
  *                           errors of the library's side streams (GPTQ_ERR_CUDA).
  *   GPTQ_FLAG_IL_FP64       accepted for compatibility: the intrinsic-LoRA path always forms its
  *                           cancelling products (Gram matrices, Schur complement) with fp64
- *                           accumulation. */
+ *                           accumulation.
+ *   GPTQ_FLAG_KERNEL_TIMES  note the device time of every fp32 GEMM launch (gptq_kernel_times). */
 typedef enum {
     GPTQ_FLAG_SYNC_STATUS = 1u,
     GPTQ_FLAG_DEBUG_CHECKS = 2u,
-    GPTQ_FLAG_IL_FP64 = 4u
+    GPTQ_FLAG_IL_FP64 = 4u,
+    GPTQ_FLAG_KERNEL_TIMES = 8u
 } gptq_flag;
 
 GPTQ_API void gptq_set_flags(unsigned flags);
@@ -106,6 +108,44 @@ GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info);
  * A diagnostic for tracing and benchmarking: the difference of two readings counts the
  * kernels a span of calls launched. Library-internal memsets are not counted. */
 GPTQ_API uint64_t gptq_launch_count(void);
+
+/* Device time of the library's fp32 GEMM launches, a benchmarking diagnostic.
+ * While GPTQ_FLAG_KERNEL_TIMES is set, every launch of the fp32 GEMM (the tf32 x 3 tensor-core
+ * kernel and the SIMT kernel) is bracketed by two CUDA events on its stream and noted with the
+ * stage that issued it and its algorithmic work. The events also order launches that would
+ * otherwise overlap a predecessor's tail, so a pass run with the flag is a little slower.
+ *
+ * gptq_kernel_times waits for every noted launch to finish, writes the totals of the first
+ * n_out classes to out[0 .. n_out) (class index = stage * 2 + path; path 0 = tensor core,
+ * 1 = SIMT; stage = gptq_kt_stage), clears the record, and returns the number of classes
+ * (GPTQ_KT_NCLASSES) or GPTQ_ERR_ARG (out NULL with n_out > 0, n_out < 0) or GPTQ_ERR_CUDA.
+ * Records of launches on a device other than the current one are read as well.
+ *   launches  number of launches
+ *   ms        sum of their event-to-event durations (a launch that waits for SMs held by
+ *             another stream's kernel counts that wait)
+ *   flops     2 x the multiply-adds with both factors structurally nonzero, over the written
+ *             entries of C (triangular operands and outputs counted exactly)
+ *   bytes     each structurally nonzero operand element read once, each written element of C
+ *             stored once and loaded once when beta != 0 */
+typedef enum {
+    GPTQ_KT_OTHER = 0,
+    GPTQ_KT_FACTOR = 1, /* blocked UL factor and inverse (gptq_prepare_hinv, the 2D factors) */
+    GPTQ_KT_SWEEP = 2,  /* lazy trailing updates of the column sweep */
+    GPTQ_KT_IL = 3,     /* intrinsic-LoRA products (Gram, subspace iteration, Schur complement) */
+    GPTQ_KT_REFINE = 4, /* OLrC + Bid-Up products */
+    GPTQ_KT_2D = 5,     /* two-sided rounding (its own products) */
+    GPTQ_KT_NSTAGES = 6
+} gptq_kt_stage;
+#define GPTQ_KT_NCLASSES 12
+
+typedef struct {
+    int64_t launches;
+    double ms;
+    double flops;
+    double bytes;
+} gptq_kernel_time;
+
+GPTQ_API int gptq_kernel_times(gptq_kernel_time *out, int n_out);
 
 /*
  * H += 2 X^T X.

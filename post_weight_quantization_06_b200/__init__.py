@@ -21,11 +21,22 @@ GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
 GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND = 4, 5
 GPTQ_FLAG_SYNC_STATUS, GPTQ_FLAG_DEBUG_CHECKS, GPTQ_FLAG_IL_FP64 = 1, 2, 4
+GPTQ_FLAG_KERNEL_TIMES = 8
+KT_STAGES = ("other", "factor", "sweep", "il", "refine", "2d")   # gptq_kt_stage order
+KT_PATHS = ("tc", "simt")
+GPTQ_KT_NCLASSES = len(KT_STAGES) * len(KT_PATHS)
 
 EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
             "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-            "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags")
+            "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags",
+            "gptq_kernel_times")
+
+
+class KernelTime(ctypes.Structure):
+    """gptq_kernel_time: totals of one class of GEMM launches."""
+    _fields_ = [("launches", ctypes.c_int64), ("ms", ctypes.c_double),
+                ("flops", ctypes.c_double), ("bytes", ctypes.c_double)]
 
 
 class GptqError(RuntimeError):
@@ -61,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "gptq_2d_round": (c_int, [c_p, c_i64, c_i64, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
         "gptq_set_flags": (None, [ctypes.c_uint]),
         "gptq_get_flags": (ctypes.c_uint, []),
+        "gptq_kernel_times": (c_int, [ctypes.POINTER(KernelTime), c_int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -122,6 +134,26 @@ def gptq_set_flags(flags: int) -> None:
 
 def gptq_get_flags() -> int:
     return int(_lib.gptq_get_flags())
+
+
+def gptq_kernel_times(out, n_out: int) -> int:
+    return int(_lib.gptq_kernel_times(out, int(n_out)))
+
+
+def kernel_times() -> dict:
+    """Reads and clears the GEMM launch record of GPTQ_FLAG_KERNEL_TIMES: {(stage, path):
+    {launches, ms, flops, bytes}} for every class with at least one launch."""
+    arr = (KernelTime * GPTQ_KT_NCLASSES)()
+    st = gptq_kernel_times(arr, GPTQ_KT_NCLASSES)
+    if st < 0:
+        raise GptqError(st, "gptq_kernel_times")
+    out = {}
+    for c in range(GPTQ_KT_NCLASSES):
+        if arr[c].launches:
+            out[(KT_STAGES[c // 2], KT_PATHS[c % 2])] = {
+                "launches": int(arr[c].launches), "ms": arr[c].ms, "flops": arr[c].flops,
+                "bytes": arr[c].bytes}
+    return out
 
 
 def gptq_launch_count() -> int:

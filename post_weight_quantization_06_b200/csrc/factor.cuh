@@ -480,6 +480,7 @@ inline FactorStreams *factor_streams(int slot) {
 // the previous block before its look-ahead; the inverse stream trails both.
 inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n, float *T,
                              cudaStream_t s, int slot = 0) {
+    KtStageScope stage(GPTQ_KT_FACTOR);
     if (n <= FACTOR_NB) return leaf_ul_inv(A, lda, U, ldu, n, 0, s);
     FactorStreams *fs = factor_streams(slot);
     if (!fs) return GPTQ_ERR_CUDA;

@@ -4,6 +4,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ktimes.cuh"
 
 namespace gptq {
 
@@ -161,12 +162,17 @@ template <typename TA, typename TB>
 inline int gemm_simt(const GemmArgs<TA, TB> &p, cudaStream_t s) {
     if (p.M <= 0 || p.N <= 0) return GPTQ_OK;
     // fewer than ~one 128-tile wave: use 64 x 64 tiles for four times the CTAs
+    KtSpan span(s);
+    int st;
     if ((long long)ceil_div(p.M, 128) * ceil_div(p.N, 128) < 148) {
         dim3 grid(ceil_div(p.N, 64), ceil_div(p.M, 64));
-        return launch_kernel(gemm_simt_kernel<TA, TB, 64>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
+        st = launch_kernel(gemm_simt_kernel<TA, TB, 64>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
+    } else {
+        dim3 grid(ceil_div(p.N, 128), ceil_div(p.M, 128));
+        st = launch_kernel(gemm_simt_kernel<TA, TB, 128>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
     }
-    dim3 grid(ceil_div(p.N, 128), ceil_div(p.M, 128));
-    return launch_kernel(gemm_simt_kernel<TA, TB, 128>, grid, dim3(simt::NT), 0, s, p.pdl != 0, p);
+    span.done(KT_SIMT, p);
+    return st;
 }
 
 template <typename TA, typename TB>

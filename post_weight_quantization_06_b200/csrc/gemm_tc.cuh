@@ -52,6 +52,8 @@ constexpr int STAGES = 3;
 constexpr int SLICE_BYTES = TILE * BK * 4;          // 16 KB
 constexpr int STAGE_BYTES = 4 * SLICE_BYTES;        // A, A_lo, B, B_lo
 constexpr int CONV_WARPS = 4, EPI_WARPS = 4;
+constexpr int CONV_PER = SLICE_BYTES / 16 / (CONV_WARPS * 32);   // float4 per converter thread
+static_assert(CONV_PER * CONV_WARPS * 32 * 16 == SLICE_BYTES, "converter threads tile a slice");
 constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
 constexpr int TMEM_COLS = 2 * TILE;
 constexpr size_t EPI_STAGE_BYTES = (size_t)EPI_WARPS * 32 * 33 * 4;
@@ -161,6 +163,19 @@ __device__ __forceinline__ void tile_of(const TcGemmParams &p, int t, int &ti, i
     tj = t % p.tiles_n;
 }
 
+// The 32 values C(row_base + r, col), r < 32, of one epilogue warp's slice (0 where C is not
+// written); all 32 reads are issued together (the compiler cannot move them across the
+// slice's stores), so a read-modify-write costs one round trip per slice.
+__device__ __forceinline__ void epi_load_c(const TcGemmParams &p, int row_base, int col,
+                                           float (&cin)[32]) {
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+        const int row = row_base + r;
+        const bool ok = row < p.M && col < p.N && !(p.c_upper && col < row);
+        cin[r] = ok ? p.C[(long long)row * p.ldc + col] : 0.f;
+    }
+}
+
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                TcGemmParams p) {
@@ -181,6 +196,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = num_tiles(p);
     if (threadIdx.x == 0) {
+        // the descriptors' first fetch overlaps the setup instead of the first TMA load
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&amap)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&bmap)) : "memory");
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&conv[s], CONV_WARPS);
@@ -304,16 +322,27 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     break;
                 }
                 unsigned char *st = base + slot * STAGE_BYTES;
+                // every thread splits CONV_PER float4 of each operand; all of its shared-memory
+                // loads go out first so that their latencies overlap
+                float4 x[2][CONV_PER];
+#pragma unroll
+                for (int op = 0; op < 2; ++op) {
+                    const float4 *hi = reinterpret_cast<const float4 *>(st + op * 2 * SLICE_BYTES);
+#pragma unroll
+                    for (int u = 0; u < CONV_PER; ++u) x[op][u] = hi[cw * 32 + lane + u * CONV_WARPS * 32];
+                }
 #pragma unroll
                 for (int op = 0; op < 2; ++op) {
                     float4 *hi = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES);
                     float4 *lo = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES + SLICE_BYTES);
-                    for (int i = cw * 32 + lane; i < SLICE_BYTES / 16; i += CONV_WARPS * 32) {
-                        const float4 x = hi[i];
+#pragma unroll
+                    for (int u = 0; u < CONV_PER; ++u) {
+                        const int i = cw * 32 + lane + u * CONV_WARPS * 32;
+                        const float4 v = x[op][u];
                         float4 h, l;
-                        h.x = to_tf32(x.x); h.y = to_tf32(x.y); h.z = to_tf32(x.z); h.w = to_tf32(x.w);
-                        l.x = to_tf32(x.x - h.x); l.y = to_tf32(x.y - h.y);
-                        l.z = to_tf32(x.z - h.z); l.w = to_tf32(x.w - h.w);
+                        h.x = to_tf32(v.x); h.y = to_tf32(v.y); h.z = to_tf32(v.z); h.w = to_tf32(v.w);
+                        l.x = to_tf32(v.x - h.x); l.y = to_tf32(v.y - h.y);
+                        l.z = to_tf32(v.z - h.z); l.w = to_tf32(v.w - h.w);
                         lo[i] = l;
                         hi[i] = h;
                     }
@@ -327,6 +356,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     } else {
         // epilogue: C = alpha * acc + beta * C
         const int q = warp & 3;
+        const bool rd = p.beta != 0.f;
+        float *stage = epi_stage + (warp - 2 - CONV_WARPS) * 32 * 33;
         long long ch = 0;
         for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
             int ti, tj;
@@ -334,6 +365,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             int kb, ke;
             tile_k_range(p, ti, tj, kb, ke);
             const bool has_acc = ke > kb;
+            // Each warp owns rows [32 q, 32 q + 32) of the tile. Per 32-column slice the values
+            // (one row per lane) pass through a padded shared buffer so that the global
+            // accesses are whole 128-byte row segments.
+            const int row_base = ti * TILE + 32 * q;
+            // C is read ahead of the accumulator: the warp's rows of the tile are requested
+            // into L2 and the first slice's values into registers before the wait, and each
+            // later slice's values right after the previous slice's stores
+            float cin[32];
+            if (rd) {
+                const int prow = row_base + lane;
+                if (prow < p.M) {
+#pragma unroll
+                    for (int c = 0; c < TILE / 32; ++c) {
+                        const int pcol = tj * TILE + 32 * c;
+                        if (pcol < p.N)
+                            asm volatile("prefetch.global.L2 [%0];" ::"l"(p.C + (long long)prow * p.ldc + pcol));
+                    }
+                }
+                epi_load_c(p, row_base, tj * TILE + lane, cin);
+            }
             int b = 0;
             if (has_acc) {
                 b = (int)(ch & 1);
@@ -344,11 +395,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 }
                 tc_fence_after();
             }
-            // Each warp owns rows [32 q, 32 q + 32) of the tile. Per 32-column slice the values
-            // (one row per lane) pass through a padded shared buffer so that the global
-            // accesses are whole 128-byte row segments.
-            float *stage = epi_stage + (warp - 2 - CONV_WARPS) * 32 * 33;
-            const int row_base = ti * TILE + 32 * q;
 #pragma unroll 1
             for (int c32 = 0; c32 < TILE / 32; ++c32) {
                 float v[32];
@@ -362,25 +408,15 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
                 __syncwarp();
                 const int col = tj * TILE + 32 * c32 + lane;
-                // all 32 reads of C are issued before any write (the compiler cannot reorder
-                // them across the stores itself), so the read-modify-write costs one round trip
-                float cin[32];
-                if (p.beta != 0.f) {
-#pragma unroll
-                    for (int r = 0; r < 32; ++r) {
-                        const int row = row_base + r;
-                        const bool ok = row < p.M && col < p.N && !(p.c_upper && col < row);
-                        cin[r] = ok ? p.C[(long long)row * p.ldc + col] : 0.f;
-                    }
-                }
 #pragma unroll
                 for (int r = 0; r < 32; ++r) {
                     const int row = row_base + r;
                     if (row >= p.M || col >= p.N || (p.c_upper && col < row)) continue;
                     const float o = p.alpha * stage[r * 33 + lane];
-                    p.C[(long long)row * p.ldc + col] = p.beta == 0.f ? o : fmaf(p.beta, cin[r], o);
+                    p.C[(long long)row * p.ldc + col] = rd ? fmaf(p.beta, cin[r], o) : o;
                 }
                 __syncwarp();
+                if (rd && c32 + 1 < TILE / 32) epi_load_c(p, row_base, col + 32, cin);
             }
             if (has_acc) {
                 tc_fence_before();
@@ -464,8 +500,11 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
     cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tcg::SMEM_BYTES);
+    KtSpan span(s);
     tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, p);
-    return launch_status();
+    const int st = launch_status();
+    span.done(KT_TC, g);
+    return st;
 }
 
 }  // namespace gptq

@@ -274,14 +274,39 @@ GPTQ_API int gptq_sync_status(gptq_stream_t stream, int64_t *info) {
     return st.code;
 }
 
-static std::atomic<unsigned> g_flags{0};
+GPTQ_API void gptq_set_flags(unsigned flags) { flags_word().store(flags); }
+GPTQ_API unsigned gptq_get_flags(void) { return flags_word().load(); }
 
-GPTQ_API void gptq_set_flags(unsigned flags) { g_flags.store(flags); }
-GPTQ_API unsigned gptq_get_flags(void) { return g_flags.load(); }
+GPTQ_API int gptq_kernel_times(gptq_kernel_time *out, int n_out) {
+    if (n_out < 0 || (n_out > 0 && !out)) return GPTQ_ERR_ARG;
+    std::vector<KtRecord> recs;
+    {
+        std::lock_guard<std::mutex> lk(kt_log().mu);
+        recs.swap(kt_log().recs);
+    }
+    gptq_kernel_time tot[GPTQ_KT_NCLASSES] = {};
+    int st = GPTQ_OK;
+    for (const KtRecord &r : recs) {
+        float ms = 0.f;
+        if (st == GPTQ_OK && (cudaEventSynchronize(r.stop) != cudaSuccess ||
+                              cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess))
+            st = GPTQ_ERR_CUDA;
+        cudaEventDestroy(r.start);
+        cudaEventDestroy(r.stop);
+        if (st != GPTQ_OK || r.cls < 0 || r.cls >= GPTQ_KT_NCLASSES) continue;
+        tot[r.cls].launches += 1;
+        tot[r.cls].ms += ms;
+        tot[r.cls].flops += r.flops;
+        tot[r.cls].bytes += r.bytes;
+    }
+    if (st != GPTQ_OK) return st;
+    for (int c = 0; c < n_out && c < GPTQ_KT_NCLASSES; ++c) out[c] = tot[c];
+    return GPTQ_KT_NCLASSES;
+}
 
 // Applied to the status of every compute entry point once its work is enqueued.
 static int finish_call(int st, gptq_stream_t stream) {
-    const unsigned f = g_flags.load();
+    const unsigned f = flags_word().load();
     if (st != GPTQ_OK || !(f & (GPTQ_FLAG_SYNC_STATUS | GPTQ_FLAG_DEBUG_CHECKS))) return st;
     if ((f & GPTQ_FLAG_DEBUG_CHECKS) &&
         (cudaDeviceSynchronize() != cudaSuccess || cudaGetLastError() != cudaSuccess))

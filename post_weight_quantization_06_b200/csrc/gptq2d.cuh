@@ -540,6 +540,7 @@ inline int gptq2d_band() {
 // The wavefront: tile anti-diagonals in bands of W; after each band that has a successor, its
 // flush into all later tiles.
 inline int gptq2d_sweep(Gptq2dArgs a, cudaStream_t s) {
+    KtStageScope stage(GPTQ_KT_2D);
     const int W = gptq2d_band();
     const int Smax = a.MT + a.NT - 2;
     const size_t smem = gptq2d_sweep_smem(W);

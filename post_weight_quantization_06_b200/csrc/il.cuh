@@ -236,6 +236,7 @@ inline int cholqr_f64(const float *src, float *dst, int n, int p, ILWork &w, cud
 // Top-r eigenvectors of H (n x n) into V (n x r).
 inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V, ILWork &w,
                           cudaStream_t s) {
+    KtStageScope stage(GPTQ_KT_IL);
     const int p = il_block_p(n, r);
     random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
     GPTQ_CHECK_LAUNCH();
@@ -275,6 +276,7 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
 inline int il_factor(const float *H, long long ldh, int n, int r, const float *V,
                      float lambda_rel, float *Uaug, float *Awork, float *T, float *lam,
                      ILWork &w, cudaStream_t s) {
+    KtStageScope stage(GPTQ_KT_IL);
     const long long ldu = n + r;
     // B12 = H V (n x r), C = V^T B12 (r x r)
     if (int st = gemm_f64acc<float, float, double>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.0,

@@ -306,6 +306,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
                        long long ldu, int bits, int group_size, int B, uint32_t *codes,
                        float *scales, uint8_t *zeros, double *loss, float *Err,
                        cudaStream_t s) {
+    KtStageScope stage(GPTQ_KT_SWEEP);
     const int gs = group_size ? group_size : n;
     const int OB = outer_block(n, gs, B);
     ColloopArgs a;

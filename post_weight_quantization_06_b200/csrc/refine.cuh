@@ -269,6 +269,7 @@ template <typename TW>
 inline int il_refine(const TW *W, int m, int n, const float *H, int r, int bits, int gs,
                      int iters, const float *scales, const uint8_t *zeros, float *L, float *R,
                      double *loss_hist, RefineWs &w, cudaStream_t s) {
+    KtStageScope stage(GPTQ_KT_REFINE);
     const int G = n / gs;
     const long long mn = (long long)m * n;
     const int blocks = (int)std::min<long long>((mn + 255) / 256, 148LL * 8);

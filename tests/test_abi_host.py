@@ -21,7 +21,8 @@ def test_header_declares_the_boundary():
         "gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gptq_launch_count",
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
         "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
-        "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags"])
+        "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags",
+        "gptq_kernel_times"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -203,3 +204,21 @@ def test_flags_round_trip_and_host_errors_stay_synchronous():
     finally:
         g.gptq_set_flags(0)
     assert g.gptq_get_flags() == 0
+
+
+def test_kernel_times_record_is_empty_and_checks_its_arguments():
+    """Nothing launched: every class reads zero (no device call is needed to read an empty
+    record); the class count and the stage names agree with the header."""
+    import post_weight_quantization_06_b200 as g
+    src = open(os.path.join(ROOT, "include", "gptq.h")).read()
+    assert f"#define GPTQ_KT_NCLASSES {g.GPTQ_KT_NCLASSES}" in src
+    stages = re.findall(r"GPTQ_KT_(\w+) = (\d+)", src)
+    names = {int(v): k.lower() for k, v in stages if k != "NSTAGES"}
+    assert tuple(names[i] for i in range(len(names))) == g.KT_STAGES
+    arr = (g.KernelTime * g.GPTQ_KT_NCLASSES)()
+    assert g.gptq_kernel_times(arr, g.GPTQ_KT_NCLASSES) == g.GPTQ_KT_NCLASSES
+    assert all(c.launches == 0 and c.ms == 0 and c.flops == 0 for c in arr)
+    assert g.gptq_kernel_times(None, 0) == g.GPTQ_KT_NCLASSES
+    assert g.gptq_kernel_times(None, 3) == g.GPTQ_ERR_ARG
+    assert g.gptq_kernel_times(arr, -1) == g.GPTQ_ERR_ARG
+    assert g.kernel_times() == {}

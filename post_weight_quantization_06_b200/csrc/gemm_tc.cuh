@@ -56,8 +56,13 @@ constexpr int CONV_PER = SLICE_BYTES / 16 / (CONV_WARPS * 32);   // float4 per c
 static_assert(CONV_PER * CONV_WARPS * 32 * 16 == SLICE_BYTES, "converter threads tile a slice");
 constexpr int THREADS = 32 * (2 + CONV_WARPS + EPI_WARPS);
 constexpr int TMEM_COLS = 2 * TILE;
-constexpr size_t EPI_STAGE_BYTES = (size_t)EPI_WARPS * 32 * 33 * 4;
-constexpr size_t SMEM_BYTES = 1024 + (size_t)STAGES * STAGE_BYTES + 256 + EPI_STAGE_BYTES;
+// Per epilogue warp: a padded 32 x 33 staging slice (read-modify-write epilogue) or one 32 x 32
+// slice in the 128-byte swizzle for the C tensor map; 1024-byte aligned for the swizzle.
+constexpr size_t EPI_WARP_BYTES = 5120;
+constexpr size_t EPI_OFFSET = (size_t)STAGES * STAGE_BYTES + 1024;   // after the barriers
+constexpr size_t SMEM_BYTES = 1024 + EPI_OFFSET + (size_t)EPI_WARPS * EPI_WARP_BYTES;
+static_assert(EPI_WARP_BYTES % 1024 == 0 && EPI_WARP_BYTES >= 32 * 33 * 4, "epilogue buffer");
+static_assert(SMEM_BYTES <= 232448, "fits the opt-in shared memory of one CTA");
 
 __host__ __device__ constexpr uint32_t idesc_tf32(int a_mn, int b_mn) {
     return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
@@ -130,7 +135,31 @@ struct TcGemmParams {
     int c_upper, a_upper, a_lower, b_upper, b_lower;
     int tiles_m, tiles_n;
     long long wait_limit;
+    int c_tma;          // 1: beta is 0 or 1 and cmap covers C; slices may leave by tensor store /
+                        // tensor add-reduction instead of a read-modify-write
 };
+
+// Bulk tensor writes of one 32 x 32 slice from shared memory (128-byte swizzle) through the C
+// map: a plain store (beta = 0) or an fp32 add-reduction performed in L2 (beta = 1; one
+// rounding of C + value, as the read-modify-write does).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(smem_u32(src)), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_add_2d(const CUtensorMap *map, const void *src, int x, int y) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(smem_u32(src)), "r"(x), "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the bulk operations of this thread have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // K range [kb, ke) (multiples of BK) of output tile (ti, tj).
 __device__ __forceinline__ void tile_k_range(const TcGemmParams &p, int ti, int tj, int &kb,
@@ -178,7 +207,7 @@ __device__ __forceinline__ void epi_load_c(const TcGemmParams &p, int row_base, 
 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-               TcGemmParams p) {
+               const __grid_constant__ CUtensorMap cmap, TcGemmParams p) {
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -191,7 +220,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     uint64_t *mma_done = acc_empty + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(mma_done + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    float *epi_stage = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256);
+    unsigned char *epi_base = base + EPI_OFFSET;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = num_tiles(p);
@@ -199,6 +228,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // the descriptors' first fetch overlaps the setup instead of the first TMA load
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&amap)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&bmap)) : "memory");
+        if (p.c_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&cmap)) : "memory");
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&conv[s], CONV_WARPS);
@@ -357,7 +387,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // epilogue: C = alpha * acc + beta * C
         const int q = warp & 3;
         const bool rd = p.beta != 0.f;
-        float *stage = epi_stage + (warp - 2 - CONV_WARPS) * 32 * 33;
+        unsigned char *ebuf = epi_base + (size_t)(warp - 2 - CONV_WARPS) * EPI_WARP_BYTES;
+        float *stage = reinterpret_cast<float *>(ebuf);
         long long ch = 0;
         for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
             int ti, tj;
@@ -365,15 +396,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             int kb, ke;
             tile_k_range(p, ti, tj, kb, ke);
             const bool has_acc = ke > kb;
-            // Each warp owns rows [32 q, 32 q + 32) of the tile. Per 32-column slice the values
-            // (one row per lane) pass through a padded shared buffer so that the global
-            // accesses are whole 128-byte row segments.
+            // Each warp owns rows [32 q, 32 q + 32) of the tile (TMEM lanes 32 q ...).
             const int row_base = ti * TILE + 32 * q;
-            // C is read ahead of the accumulator: the warp's rows of the tile are requested
-            // into L2 and the first slice's values into registers before the wait, and each
-            // later slice's values right after the previous slice's stores
+            // With beta 0 or 1, an accumulator and no diagonal cut, the slices leave through
+            // the C map and C is never read here; otherwise C is read and written in place.
+            const bool via_map = p.c_tma && has_acc && !(p.c_upper && ti == tj);
+            // The read-modify-write path reads C ahead of the accumulator: the warp's rows of
+            // the tile are requested into L2 and the first slice's values into registers before
+            // the wait, each later slice's values right after the previous slice's stores.
             float cin[32];
-            if (rd) {
+            if (rd && !via_map) {
                 const int prow = row_base + lane;
                 if (prow < p.M) {
 #pragma unroll
@@ -395,28 +427,57 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 }
                 tc_fence_after();
             }
+            if (via_map) {
 #pragma unroll 1
-            for (int c32 = 0; c32 < TILE / 32; ++c32) {
-                float v[32];
-                if (has_acc) {
+                for (int c32 = 0; c32 < TILE / 32; ++c32) {
+                    float v[32];
                     tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * TILE + 32 * c32), v);
-                } else {
+                    // the buffer is free once the previous slice's bulk write has read it
+                    if (lane == 0) bulk_wait_read();
+                    __syncwarp();
+                    // lane = row of the slice; 16-byte chunk c of the row sits at c ^ (row % 8)
+                    float4 *dst = reinterpret_cast<float4 *>(ebuf + lane * 128);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    for (int c = 0; c < 8; ++c)
+                        dst[c ^ (lane & 7)] = make_float4(p.alpha * v[4 * c], p.alpha * v[4 * c + 1],
+                                                          p.alpha * v[4 * c + 2], p.alpha * v[4 * c + 3]);
+                    // generic-proxy writes must be visible to the bulk copy's async proxy
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    const int x = tj * TILE + 32 * c32;
+                    if (lane == 0 && x < p.N && row_base < p.M) {
+                        if (rd) tma_add_2d(&cmap, ebuf, x, row_base);
+                        else tma_store_2d(&cmap, ebuf, x, row_base);
+                        bulk_commit();
+                    }
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
+            } else {
+                // a bulk write of an earlier tile may still be reading the shared buffer
+                if (lane == 0) bulk_wait_read();
                 __syncwarp();
-                const int col = tj * TILE + 32 * c32 + lane;
+#pragma unroll 1
+                for (int c32 = 0; c32 < TILE / 32; ++c32) {
+                    float v[32];
+                    if (has_acc) {
+                        tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * TILE + 32 * c32), v);
+                    } else {
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    const int row = row_base + r;
-                    if (row >= p.M || col >= p.N || (p.c_upper && col < row)) continue;
-                    const float o = p.alpha * stage[r * 33 + lane];
-                    p.C[(long long)row * p.ldc + col] = rd ? fmaf(p.beta, cin[r], o) : o;
+                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) stage[lane * 33 + i] = v[i];
+                    __syncwarp();
+                    const int col = tj * TILE + 32 * c32 + lane;
+#pragma unroll
+                    for (int r = 0; r < 32; ++r) {
+                        const int row = row_base + r;
+                        if (row >= p.M || col >= p.N || (p.c_upper && col < row)) continue;
+                        const float o = p.alpha * stage[r * 33 + lane];
+                        p.C[(long long)row * p.ldc + col] = rd ? fmaf(p.beta, cin[r], o) : o;
+                    }
+                    __syncwarp();
+                    if (rd && c32 + 1 < TILE / 32) epi_load_c(p, row_base, col + 32, cin);
                 }
-                __syncwarp();
-                if (rd && c32 + 1 < TILE / 32) epi_load_c(p, row_base, col + 32, cin);
             }
             if (has_acc) {
                 tc_fence_before();
@@ -425,6 +486,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 ++ch;
             }
         }
+        // every bulk write is complete before the CTA (and its shared memory) goes away
+        if (lane == 0) bulk_wait_all();
+        __syncwarp();
     }
     tc_fence_before();
     __syncthreads();
@@ -486,12 +550,18 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     p.tiles_m = ceil_div(g.M, tcg::TILE);
     p.tiles_n = ceil_div(g.N, tcg::TILE);
     p.wait_limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
-    CUtensorMap am, bm;
+    CUtensorMap am, bm, cm;
     const bool ok_a = p.a_mn ? tcg::make_map_f32(&am, g.A, g.K, g.M, g.lda, 32, 32, true)
                              : tcg::make_map_f32(&am, g.A, g.M, g.K, g.lda, 32, tcg::TILE, false);
     const bool ok_b = p.b_mn ? tcg::make_map_f32(&bm, g.B, g.K, g.N, g.ldb, 32, 32, true)
                              : tcg::make_map_f32(&bm, g.B, g.N, g.K, g.ldb, 32, tcg::TILE, false);
     if (!ok_a || !ok_b) return gemm_simt(g, s);
+    // C through a tensor map when beta is 0 or 1 and C's base and pitch allow it
+    static const bool rmw_only = std::getenv("GPTQ_GEMM_RMW_EPILOGUE") != nullptr;
+    p.c_tma = !rmw_only && (g.beta == 0.f || g.beta == 1.f) &&
+              (reinterpret_cast<uintptr_t>(g.C) & 15u) == 0 && g.ldc % 4 == 0 &&
+              tcg::make_map_f32(&cm, g.C, g.M, g.N, g.ldc, 32, 32, false);
+    if (!p.c_tma) cm = am;   // not read
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -501,7 +571,7 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)tcg::SMEM_BYTES);
     KtSpan span(s);
-    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, p);
+    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, cm, p);
     const int st = launch_status();
     span.done(KT_TC, g);
     return st;

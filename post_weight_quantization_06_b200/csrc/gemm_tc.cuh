@@ -15,7 +15,9 @@
 //   warp 0     TMA producer, 3-stage ring of {A, A_lo, B, B_lo} (64 KB per stage)
 //   warp 1     TMEM allocation and the MMA issuer (one thread); 3 x 4 MMAs per stage
 //   warps 2-5  hi/lo converters
-//   warps 6-9  epilogue: one row of the tile per thread (TMEM lane = row)
+//   warps 6-9  epilogue: one row of the tile per thread (TMEM lane = row); per 32-column
+//              slice either a bulk tensor store / add-reduction of alpha * acc through the C
+//              map (beta 0 or 1) or a read-modify-write of C through shared memory
 // Triangular operands: a_upper / a_lower / b_upper / b_lower restrict each tile's K range to
 // where the operand can be nonzero; the storage of the zero triangle must hold zeros.
 // All mbarrier waits are bounded as in the Hessian kernel.

@@ -106,8 +106,10 @@ def test_hessian_bounded_wait_reports_timeout_and_device_stays_usable(g, monkeyp
 
 # ----------------------------------------------------------------------------- factor
 
+# n = 1000: the factor's tensor-core updates have widths that are not multiples of 32 (their
+# last 32-column slices cross the matrix edge)
 @pytest.mark.parametrize("n,k,lam", [(256, 512, 0.01), (300, 2000, 0.01), (1024, 4096, 0.01),
-                                     (129, 400, 0.1)])
+                                     (129, 400, 0.1), (1000, 3000, 0.01)])
 def test_prepare_hinv_matches_oracle(g, n, k, lam):
     X = _spd_from_data(n, k, 7 * n)
     H32 = oracle.hessian(X).astype(np.float32)
@@ -202,6 +204,8 @@ SWEEP_CASES = [
     (48, 256, 5, 64, 64, torch.float32),
     (40, 512, 6, 128, 128, torch.bfloat16),
     (36, 256, 7, 32, 32, torch.float32),
+    # 300 rows: the tensor-core lazy updates' last 32-row slices cross the matrix edge
+    (300, 640, 4, 128, 128, torch.float32),
     # several 1024-column outer blocks of the two-level lazy update
     (64, 2560, 3, 128, 128, torch.bfloat16),
     (40, 2048, 4, 0, 128, torch.float32),

@@ -216,6 +216,32 @@ def hessian_flops(layer) -> float:
     return float(layer.k) * layer.n * (layer.n + 1)
 
 
+def sweep_bytes(layer) -> float:
+    """Algorithmic bytes of the sweep stage: W read once (its stored dtype), the upper triangle
+    of U read once, the packed codes, and the per-group scales (fp32) and zero-points (u8)."""
+    m, n = layer.m, layer.n
+    groups = n // layer.group_size if layer.group_size else 1
+    w_bytes = layer.W.element_size()
+    return float(m * n * w_bytes + 4 * n * (n + 1) // 2 + m * n * layer.bits // 8 + m * groups * 5)
+
+
+def sweep_roofline(layer, sweep_ms: float, gemm) -> dict:
+    """The sweep against HBM: its algorithmic bytes over the timed stage. The stage is bound by
+    its n sequential column steps, not by bandwidth, so the fraction is small by design; with
+    the GEMM timing pass, the column loops' own share is the stage time minus the event time of
+    the sweep's GEMM launches (two passes of the same code)."""
+    hbm = hbm_peak_gbs()
+    b = sweep_bytes(layer)
+    gbs = b / (sweep_ms * 1e-3) / 1e9
+    out = {"bound": "latency (n sequential column steps)", "bytes": b, "achieved_gbs": gbs,
+           "peak_gbs": hbm, "frac": gbs / hbm, "peak_source": "measured copy (MEASURED_PEAKS.json)"}
+    if gemm:
+        g_ms = sum(v["ms"] for k, v in gemm.items() if k.startswith("sweep_") and isinstance(v, dict))
+        out["gemm_ms"] = g_ms
+        out["column_loop_ms"] = max(sweep_ms - g_ms, 0.0)
+    return out
+
+
 def hessian_traffic(layer):
     """DRAM bytes per Hessian launch from the committed ncu summary, for the full 2048x6144 /
     262144-token workload only, and only while the kernel source is the one profiled."""
@@ -600,6 +626,7 @@ def bench_ours(args):
         }
         if e2e:
             out["e2e"] = e2e
+        out["sweep_roofline"] = sweep_roofline(layer, float(stage[2]), gemm)
         if gemm:
             out["gemm"] = gemm
         if refine:

@@ -57,3 +57,21 @@ def test_reduce_max_over_two_gloo_ranks():
 
 def test_reduce_max_single_process_is_identity():
     assert bench.reduce_max(3.25, "cpu") == 3.25
+
+
+def test_sweep_bytes_and_roofline():
+    """Sweep bytes of the 2048 x 6144 bf16 layer at 3 bits, groups of 128: W 25.2 MB, the upper
+    triangle of U 75.5 MB, codes 4.7 MB, scales and zero-points 0.49 MB; the GEMM share is
+    subtracted from the stage time."""
+    from types import SimpleNamespace
+    W = torch.empty(2048, 6144, dtype=torch.bfloat16)
+    layer = SimpleNamespace(m=2048, n=6144, W=W, bits=3, group_size=128)
+    b = bench.sweep_bytes(layer)
+    assert b == 2048 * 6144 * 2 + 4 * 6144 * 6145 // 2 + 2048 * 6144 * 3 // 8 + 2048 * 48 * 5
+    assert abs(b / 1e6 - 105.9) < 0.1
+    r = bench.sweep_roofline(layer, 2.0, {"sweep_tc": {"ms": 1.25}, "factor_tc": {"ms": 4.0},
+                                          "peak_tc": 229.0})
+    assert abs(r["achieved_gbs"] - b / 2e-3 / 1e9) < 1e-9
+    assert r["gemm_ms"] == 1.25 and abs(r["column_loop_ms"] - 0.75) < 1e-12
+    assert 0 < r["frac"] < 1
+    assert "gemm_ms" not in bench.sweep_roofline(layer, 2.0, None)

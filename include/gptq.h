@@ -12,6 +12,7 @@
  *   gptq_quantize_lowrank     L and R stored at low precision (4-bit L, 8-bit R) on min-max grids
  *   gptq_2d_round             two-sided adaptive rounding of a real matrix to integers (GPTQ-2D)
  *   gptq_set_flags            synchronous status returns and debug synchronisation (see below)
+ *   gptq_kernel_times         device time and algorithmic work of the GEMM launches (diagnostic)
  *
  * Conventions shared by every entry point
  *   - Orientation: W is m x n row-major (m output rows, n input columns: one neuron per row);

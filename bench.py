@@ -58,6 +58,10 @@ def parse_args(argv=None):
                     help="time only the two-sided rounding (one GPU) and print its JSON object")
     ap.add_argument("--tokens", type=int, default=0,
                     help="use only the first TOKENS calibration rows (small profiling cases)")
+    ap.add_argument("--no-il", action="store_true",
+                    help="skip the intrinsic-LoRA layer pass reported under 'il'")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads (tiny, attn, DeiT fc1/fc2) reported under 'configs'")
     return ap.parse_args(argv)
 
 
@@ -476,6 +480,68 @@ def run_gptq2d(g, dev, steps):
                          "peak_source": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz"}}
 
 
+def config_dict(layer, world: int = 1) -> dict:
+    """The workload as both arms report it."""
+    return {"workload": layer.name, "m": layer.m, "n": layer.n, "k_tokens": layer.k,
+            "bits": layer.bits, "group_size": layer.group_size, "r": layer.r,
+            "block_size": layer.block_size, "lambda_rel": layer.lambda_rel,
+            "l2": "inputs larger than L2 (X is %.1f GB)" % (layer.X.numel() * layer.X.element_size() / 1e9)
+            if layer.X.numel() * layer.X.element_size() > 126e6 else
+            "inputs smaller than L2 (X is %.1f MB)" % (layer.X.numel() * layer.X.element_size() / 1e6),
+            "parallelism": f"{world} independent layers (one per GPU)"}
+
+
+def time_workload(g, layer, steps: int, warmup: int) -> dict:
+    """One workload's whole layer pass (H = 0, Hessian over all tokens, factor or
+    intrinsic-LoRA step, sweep) timed like the main step: CUDA events on the launching stream,
+    `warmup` untimed passes first. Reported apart from the main line."""
+    dev = layer.W.device
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.Stream(device=dev)
+    lp = LayerPass(g, layer, s)
+    for _ in range(warmup):
+        lp.step()
+    torch.cuda.synchronize(dev)
+    g.gptq_sync_status(s)
+    events = [LayerPass.new_events() for _ in range(steps)]
+    l0 = g.gptq_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s)
+    for i in range(steps):
+        lp.step(events[i])
+    e1.record(s)
+    torch.cuda.synchronize(dev)
+    launches = (g.gptq_launch_count() - l0) // max(1, steps)
+    stage = np.zeros(3)
+    for ev in events:
+        lp.ev = ev
+        stage += np.array(lp.stage_ms())
+    stage /= steps
+    ms = e0.elapsed_time(e1) / steps
+    st, info = g.gptq_sync_status(s, raise_on_error=False)
+    out = {"config": config_dict(layer), "ms": ms, "weights_per_s": layer.m * layer.n / (ms * 1e-3),
+           "steps": steps, "launches_per_step": int(launches), "device_status": int(st)}
+    if layer.r:
+        out["stages_ms"] = {"hessian": stage[0], "il_quantize": stage[2]}
+    else:
+        out["stages_ms"] = {"hessian": stage[0], "factor": stage[1], "sweep": stage[2]}
+    out["hessian_tflops"] = hessian_flops(layer) / (stage[0] * 1e-3) / 1e12
+    del lp
+    return out
+
+
+def run_other_workloads(g, dev, steps: int, warmup: int, rank: int) -> dict:
+    """The other seeded workloads, one layer each, generated on the device in turn."""
+    import datagen
+    out = {}
+    for name in ("tiny", "attn", "deit_fc1", "deit_fc2"):
+        layer = datagen.WORKLOADS[name](device=dev, seed=rank_seed(name, rank))
+        out[name] = time_workload(g, layer, steps, warmup)
+        del layer
+        torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(layer, budget_s: float):
     """The fp64 oracle as it stands, on a bounded sample of the same layer, on the host cores:
     Hessian over a slice of the tokens, the full n x n factor, the sweep over a few rows;
@@ -595,6 +661,21 @@ def bench_ours(args):
         e2e = {"value": world * layer.m * layer.n / (e_ms * 1e-3), "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
+    # the other workloads, each timed on its own after the main line's measurements
+    other = None
+    il = None
+    if not args.no_configs or not args.no_il:
+        del lp
+        torch.cuda.empty_cache()
+        import datagen
+        if not args.no_il and args.workload != "lowrank":
+            il_layer = datagen.lowrank(device=dev, seed=rank_seed("lowrank", rank))
+            il = time_workload(g, il_layer, max(1, args.steps), max(1, min(args.warmup, 3)))
+            del il_layer
+            torch.cuda.empty_cache()
+        if not args.no_configs:
+            other = run_other_workloads(g, dev, max(1, args.steps), max(1, min(args.warmup, 3)), rank)
+
     if rank == 0:
         out = {
             "metric": METRIC,
@@ -609,11 +690,7 @@ def bench_ours(args):
             "vs_baseline": None,
             "dtype": "bf16 X / fp32 accumulate; fp32 factor and sweep",
             "data": "synthetic (seeded; shapes and spectra of the named layer)",
-            "config": {"workload": layer.name, "m": layer.m, "n": layer.n, "k_tokens": layer.k,
-                       "bits": layer.bits, "group_size": layer.group_size, "r": layer.r,
-                       "block_size": layer.block_size, "lambda_rel": layer.lambda_rel,
-                       "l2": "inputs larger than L2 (X is %.1f GB)" % (layer.X.numel() * 2 / 1e9),
-                       "parallelism": f"{world} independent layers (one per GPU)"},
+            "config": config_dict(layer, world),
             "stages_ms": {"hessian": stage[0], "factor": stage[1], "sweep": stage[2]},
             "roofline": {"bound": "tensor", "kernel": "hessian (2 X^T X)",
                          "achieved": h_tflops, "peak": peak, "unit": "TFLOP/s",
@@ -633,6 +710,10 @@ def bench_ours(args):
             out["refine"] = refine
         if two_d:
             out["gptq2d"] = two_d
+        if il:
+            out["il"] = il
+        if other:
+            out["configs"] = other
         if not args.no_cpu_baseline and world == 1:
             out["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
         print(json.dumps(out))
@@ -641,19 +722,25 @@ def bench_ours(args):
 
 
 def bench_reference(args):
-    """The oracle on the host cores, each step a bounded sample of the workload."""
+    """The oracle on the host cores, each step a bounded sample of the workload. ms_per_step is
+    the measured wall time of one such sample; `value` is the metric the sample gives for the
+    whole layer (per-layer time extrapolated as cpu_baseline describes, under its own key)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import datagen
     layer = datagen.WORKLOADS[args.workload](device="cuda" if torch.cuda.is_available() else "cpu",
                                               seed=rank_seed(args.workload, 0))
+    if args.tokens:
+        layer.X = layer.X[: args.tokens].clone()
     for _ in range(args.warmup):
         cpu_baseline(layer, args.cpu_budget_s)
-    vals, secs = [], []
+    vals, secs, walls = [], [], []
     t0 = time.perf_counter()
     for _ in range(args.steps):
+        t1 = time.perf_counter()
         cb = cpu_baseline(layer, args.cpu_budget_s)
+        walls.append(time.perf_counter() - t1)
         vals.append(cb["value"])
         secs.append(cb["seconds_per_layer"])
     wall = time.perf_counter() - t0
@@ -661,12 +748,13 @@ def bench_reference(args):
     print(json.dumps({
         "impl": "reference",
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": float(np.median(secs)) * 1e3,
+        "warmup": args.warmup, "ms_per_step": float(np.mean(walls)) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded; same layer as the device arm)",
-        "config": {"workload": layer.name, "m": layer.m, "n": layer.n, "k_tokens": layer.k},
+        "config": config_dict(layer),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cb["cores"], "kind": "oracle",
                          "sample": cb["sample"]},
+        "extrapolated_ms_per_layer": float(np.median(secs)) * 1e3,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "wall_s": wall,
     }))

@@ -57,7 +57,10 @@ typedef enum {
     GPTQ_ERR_NONFINITE = -3,  /* NaN or Inf in W or in diag(H) (info: the flat index) */
     GPTQ_ERR_TIMEOUT = -4,    /* a bounded device-side wait gave up (info: the site) */
     GPTQ_ERR_CUDA = -5,       /* the CUDA runtime refused a launch (see cudaGetLastError) */
-    GPTQ_ERR_WORKSPACE = -6   /* workspace pointer NULL, misaligned or too small */
+    GPTQ_ERR_WORKSPACE = -6,  /* workspace pointer NULL, misaligned or too small */
+    GPTQ_ERR_NOT_CONVERGED = -7 /* the top-r eigenvector iteration hit its cap before its
+                                   residual test passed (info: iterations run); the outputs
+                                   are those of the last iteration */
 } gptq_status;
 
 typedef enum { GPTQ_BF16 = 0, GPTQ_F32 = 1 } gptq_dtype;
@@ -229,11 +232,15 @@ GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t 
  * process exits. The caller still provides W, U and the outputs, as for
  * gptq_quantize_layer, and the arguments mean the same.
  *   - Limit: gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size) must not exceed
- *     GPTQ_NOALLOC_SCRATCH_BYTES (m * n + m * block_size floats, each part rounded up to
- *     256 bytes; e.g. 2048 x 6144 fits); larger layers get GPTQ_ERR_ARG and nothing is
- *     enqueued.
+ *     GPTQ_NOALLOC_SCRATCH_BYTES. That size is m * n floats (the working copy) plus
+ *     m * max(min(n, 1024), block_size) floats (the errors of one 1024-column outer block),
+ *     each part rounded up to 256 bytes; e.g. 2048 x 6144 fits, 2048 x 7680 does not. Larger
+ *     layers get GPTQ_ERR_ARG and nothing is enqueued.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *     with that device current; make that first call before any stream capture. The address
+ *     is tied to the device's current context: a call made after that context was destroyed
+ *     and replaced (cudaDeviceReset, or a framework that resets the device) looks it up again
+ *     (and must then come before any capture too).
  *   - Every call on a device shares the one array and leaves its contents behind. Calls
  *     whose work overlaps on the GPU (other streams, other host threads) race on it:
  *     serialise them. Nothing in the array needs to start at zero.
@@ -252,11 +259,18 @@ GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, 
  * vectors of X; the pass runs on W~ = [W, 0] (r extra zero-initialised coordinates per
  * row, placed after the n original ones and never quantized); the extra coordinates
  * absorb the quantization error and end as R; the singular augmented Hessian is factored
- * without a plain Cholesky of it. Here: V_r by subspace iteration on G = H/2 with a
- * Rayleigh-Ritz step; H~ = 2 X~^T X~ + lambda~ I with lambda~ = lambda_rel * mean of
- * the n + r diagonal entries of 2 X~^T X~; the first n rows of U~ (H~^-1 = U~^T U~)
- * come from the Schur complement of the extra block, which is positive definite.
- * With r == 0 this is gptq_prepare_hinv + gptq_quantize_layer.
+ * without a plain Cholesky of it. Here: V_r by subspace iteration on H (a block of
+ * p = min(max(r + 32, 2r), 128, n) columns): power steps with fp32-accurate tensor-core
+ * products first, then fp64-accumulated iterations, each with a Rayleigh-Ritz step, until
+ * every one of the r Ritz pairs (theta, v) has ||H v - theta v|| <= 5e-6 theta (at most 12
+ * fp64 iterations; the environment variable GPTQ_IL_MAX_ITERS, read at each call, changes
+ * the cap). If the cap is reached first the call still completes with the last iterate and
+ * the status word reports GPTQ_ERR_NOT_CONVERGED (info = iterations run). Eigenvalues that
+ * are equal at the r-th position make V_r non-unique; they are assumed distinct.
+ * H~ = 2 X~^T X~ + lambda~ I with lambda~ = lambda_rel * mean of the n + r diagonal entries
+ * of 2 X~^T X~; the first n rows of U~ (H~^-1 = U~^T U~) come from the Schur complement of
+ * the extra block, which is positive definite. With r == 0 this is gptq_prepare_hinv +
+ * gptq_quantize_layer.
  *   H          device, n x n fp32 raw Hessian 2 X^T X (from gptq_hessian_accumulate).
  *   r          0 <= r <= 128 and r < n.
  *   L          device, n x r fp32 (V_r, columns sorted by decreasing eigenvalue, each
@@ -265,7 +279,7 @@ GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, 
  *   lambda_out device, one fp32: lambda~.
  *   other arguments as in gptq_quantize_layer.
  *   workspace  device, >= gptq_workspace_size(GPTQ_OP_IL_QUANTIZE, m, n, r, block_size).
- * Device errors as in gptq_prepare_hinv and gptq_quantize_layer.
+ * Device errors as in gptq_prepare_hinv and gptq_quantize_layer, and GPTQ_ERR_NOT_CONVERGED.
  */
 GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
                            int r, int bits, int group_size, float lambda_rel, int block_size,
@@ -296,8 +310,10 @@ GPTQ_API int gptq_il_quantize_layer(const void *W, int w_dtype, int64_t m, int64
  *   loss_hist  device, 2 * iters doubles: the reconstruction error (with X^T X = H / 2)
  *              after each round's OLrC and after its Bid-Up, in order.
  *   workspace  device, >= gptq_workspace_size(GPTQ_OP_IL_REFINE, m, n, r, 0) bytes.
- * Argument errors: GPTQ_ERR_ARG, GPTQ_ERR_WORKSPACE (nothing enqueued). Device errors
- * (non-positive pivot in the eigenvector step's orthonormalisation) go to the status word.
+ * The eigenvectors come from the same iteration as in gptq_il_quantize_layer (same stopping
+ * rule and cap). Argument errors: GPTQ_ERR_ARG, GPTQ_ERR_WORKSPACE (nothing enqueued). Device
+ * errors (a non-positive pivot in the eigenvector step's orthonormalisation, an iteration that
+ * reached its cap: GPTQ_ERR_NOT_CONVERGED) go to the status word.
  */
 GPTQ_API int gptq_il_refine(const void *W, int w_dtype, int64_t m, int64_t n, const float *H,
                             int r, int bits, int group_size, int iters, uint32_t *codes,

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libgptq.so")
 
 GPTQ_OK, GPTQ_ERR_ARG, GPTQ_ERR_NOT_PD, GPTQ_ERR_NONFINITE = 0, -1, -2, -3
 GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
+GPTQ_ERR_NOT_CONVERGED = -7
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
 GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND = 4, 5

@@ -57,6 +57,38 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 
 inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
+// Multiprocessor count of the current device, looked up once per device.
+inline int device_sm_count() {
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int v = cache[dev].load(std::memory_order_relaxed);
+    if (v > 0) return v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1)
+        v = 148;
+    cache[dev].store(v, std::memory_order_relaxed);
+    return v;
+}
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current device unless this
+// call site already set at least that much there (`set_bytes` holds the value per device).
+template <typename K>
+inline void smem_limit_once(K *kernel, int bytes, std::atomic<int> *set_bytes) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (set_bytes[dev].load(std::memory_order_acquire) >= bytes) return;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+        cudaSuccess) {
+        int prev = set_bytes[dev].load();
+        while (prev < bytes && !set_bytes[dev].compare_exchange_weak(prev, bytes)) {}
+    }
+}
+#define GPTQ_SMEM_LIMIT(kernel, bytes)                                  \
+    do {                                                                \
+        static std::atomic<int> gptq_smem_set_[64];                     \
+        ::gptq::smem_limit_once(kernel, (int)(bytes), gptq_smem_set_);  \
+    } while (0)
+
 // Every kernel launch of the library is followed by launch_status(), which also counts it
 // (read with gptq_launch_count()).
 inline std::atomic<unsigned long long> &launch_counter() {

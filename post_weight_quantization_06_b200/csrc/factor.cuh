@@ -28,95 +28,108 @@ constexpr int FACTOR_NB = 128;
 // its factor. On exit U's block holds U_pp = Ubar_pp^-1 (upper; strictly lower part zeroed),
 // where A_pp = Ubar_pp Ubar_pp^T; Ubar_pp itself is used by no later step and is not stored.
 //
-// Register-tiled sweep: thread (ty, tx) of a 16 x 16 grid holds the 8 x 8 entries with rows
-// ty + 16 a and columns tx + 16 b of one matrix M. Before step c, M's columns <= c hold the
-// leading block still to be factored and its columns > c hold, for rows < c, the partial sums
-// P[i][j] = sum_{k > c} Ubar[i][k] X[k][j] of the inverse X = Ubar^-1 (rows > c of M already
-// are rows of X). Step c (from the last column to the first), with one barrier:
+// Register-tiled sweep: thread (ty, tx) of a TG x TG grid holds the TS x TS entries with rows
+// ty + TG a and columns tx + TG b of one matrix M (TG TS = 128). Before step c, M's columns <= c
+// hold the leading block still to be factored and its columns > c hold, for rows < c, the
+// partial sums P[i][j] = sum_{k > c} Ubar[i][k] X[k][j] of the inverse X = Ubar^-1 (rows > c of
+// M already are rows of X). Step c (from the last column to the first), with one barrier:
 //   column c (rows <= c) and row c (columns > c) of M are published to shared memory;
 //   pivot d = M[c][c], u_i = M[i][c] / sqrt(d) (Ubar's column c), row c of X is
 //   x_c = 1/sqrt(d), x_j = -P[c][j] / sqrt(d);
 //   rows i < c get M[i][j] += u_i v_j with v_j = -u_j (j < c: the Cholesky update),
 //   v_c = x_c (column c restarts as a partial sum), v_j = x_j (j > c: the inverse update).
 // A pivot <= 0 (or NaN) records GPTQ_ERR_NOT_PD with info = col_base + c and continues with a
-// unit pivot so that the kernel always finishes.
-constexpr int DIAG_THREADS = 256;
+// unit pivot so that the kernel always finishes. fp32 blocks use 16 x 16 threads, fp64 blocks
+// (the small Gram and extra-block factors of the intrinsic-LoRA step) 32 x 32, which shortens
+// each step's dependent chain of fp64 FMAs.
+template <typename T> struct DiagCfg { static constexpr int TG = 16, TS = 8; };
+template <> struct DiagCfg<double> { static constexpr int TG = 32, TS = 4; };
 
 template <typename T>
-__global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, long long lda,
-                                                                   T *U, long long ldu, int nb,
-                                                                   long long col_base) {
-    // wb[c' ] = M[c'][c] for c' < c (column c), -1 at c, M[c][c'] for c' > c (row c); the
+__global__ __launch_bounds__(DiagCfg<T>::TG * DiagCfg<T>::TG) void diag_ul_inv_kernel(
+    const T *A, long long lda, T *U, long long ldu, int nb, long long col_base, const int *skip) {
+    constexpr int TG = DiagCfg<T>::TG, TS = DiagCfg<T>::TS;
+    if (skip && *skip) return;
+    // wb[c'] = M[c'][c] for c' < c (column c), -1 at c, M[c][c'] for c' > c (row c); the
     // pivot M[c][c] separately. Then u_i = ipiv wb[i] (i < c) and v_j = -ipiv wb[j].
     __shared__ T wb[2][FACTOR_NB];
     __shared__ T dpiv[2];
-    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
-    T M[8][8];
+    const int tid = threadIdx.x, tx = tid % TG, ty = tid / TG;
+    T M[TS][TS];
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < TS; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int i = ty + 16 * a, j = tx + 16 * b;
+        for (int b = 0; b < TS; ++b) {
+            const int i = ty + TG * a, j = tx + TG * b;
             T v = T(0);
             if (i < nb && j < nb) v = j >= i ? A[(long long)i * lda + j] : A[(long long)j * lda + i];
             M[a][b] = v;
         }
     int buf = 0;
 #pragma unroll
-    for (int b = 7; b >= 0; --b) {
-        for (int cc = 15; cc >= 0; --cc) {
-            const int c = 16 * b + cc;
+    for (int b = TS - 1; b >= 0; --b) {
+        for (int cc = TG - 1; cc >= 0; --cc) {
+            const int c = TG * b + cc;
             if (c >= nb) continue;
             if (tx == cc) {
 #pragma unroll
-                for (int a = 0; a < 8; ++a) {
-                    const int i = ty + 16 * a;
+                for (int a = 0; a < TS; ++a) {
+                    const int i = ty + TG * a;
                     if (i < c) wb[buf][i] = M[a][b];
-                    else if (i == c) { wb[buf][c] = T(-1); dpiv[buf] = M[a][b]; }
+                    else if (i == c) {
+                        // the pivot's owner: 1/sqrt(d) (hardware estimate refined by one
+                        // Newton step), or NaN to flag a pivot <= 0 / NaN
+                        const T d = M[a][b];
+                        wb[buf][c] = T(-1);
+                        T ip = T(NAN);
+                        if (d > T(0) && isfinite((double)d)) {
+                            ip = rsqrt(d);
+                            ip = ip * (T(1.5) - T(0.5) * d * ip * ip);
+                        }
+                        dpiv[buf] = ip;
+                    }
                 }
             }
             if (ty == cc) {
 #pragma unroll
-                for (int b2 = 0; b2 < 8; ++b2) {
-                    const int j = tx + 16 * b2;
+                for (int b2 = 0; b2 < TS; ++b2) {
+                    const int j = tx + TG * b2;
                     if (j > c && j < nb) wb[buf][j] = M[b][b2];
                 }
             }
             __syncthreads();
-            const T d = dpiv[buf];
-            const bool bad = !(d > T(0)) || !isfinite((double)d);
-            if (bad && tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
-            // 1/sqrt(d): hardware estimate refined by one Newton step
-            const T dd = bad ? T(1) : d;
-            T ipiv = rsqrt(dd);
-            ipiv = ipiv * (T(1.5) - T(0.5) * dd * ipiv * ipiv);
-            T u[8], v[8];
+            T ipiv = dpiv[buf];
+            if (!(ipiv == ipiv)) {   // pivot <= 0 or NaN: report, go on with a unit pivot
+                if (tid == 0) report(GPTQ_ERR_NOT_PD, col_base + c);
+                ipiv = T(1);
+            }
+            T u[TS], v[TS];
 #pragma unroll
-            for (int a = 0; a < 8; ++a) {
-                const int i = ty + 16 * a;
+            for (int a = 0; a < TS; ++a) {
+                const int i = ty + TG * a;
                 u[a] = i < c ? wb[buf][i] * ipiv : T(0);
             }
 #pragma unroll
-            for (int b2 = 0; b2 < 8; ++b2) {
-                const int j = tx + 16 * b2;
+            for (int b2 = 0; b2 < TS; ++b2) {
+                const int j = tx + TG * b2;
                 v[b2] = j < nb ? -ipiv * wb[buf][j] : T(0);
             }
             if (tx == cc) {
 #pragma unroll
-                for (int a = 0; a < 8; ++a)
-                    if (ty + 16 * a < c) M[a][b] = T(0);
+                for (int a = 0; a < TS; ++a)
+                    if (ty + TG * a < c) M[a][b] = T(0);
             }
 #pragma unroll
-            for (int a = 0; a < 8; ++a) {
-                if (ty + 16 * a < c) {
+            for (int a = 0; a < TS; ++a) {
+                if (ty + TG * a < c) {
 #pragma unroll
-                    for (int b2 = 0; b2 < 8; ++b2) M[a][b2] = fma(u[a], v[b2], M[a][b2]);
+                    for (int b2 = 0; b2 < TS; ++b2) M[a][b2] = fma(u[a], v[b2], M[a][b2]);
                 }
             }
             if (ty == cc) {
 #pragma unroll
-                for (int b2 = 0; b2 < 8; ++b2) {
-                    const int j = tx + 16 * b2;
+                for (int b2 = 0; b2 < TS; ++b2) {
+                    const int j = tx + TG * b2;
                     if (j >= c && j < nb) M[b][b2] = v[b2];
                 }
             }
@@ -124,10 +137,10 @@ __global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, l
         }
     }
 #pragma unroll
-    for (int a = 0; a < 8; ++a)
+    for (int a = 0; a < TS; ++a)
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-            const int i = ty + 16 * a, j = tx + 16 * b;
+        for (int b = 0; b < TS; ++b) {
+            const int i = ty + TG * a, j = tx + TG * b;
             if (i < nb && j < nb) U[(long long)i * ldu + j] = j >= i ? M[a][b] : T(0);
         }
 }
@@ -135,8 +148,9 @@ __global__ __launch_bounds__(DIAG_THREADS) void diag_ul_inv_kernel(const T *A, l
 // U_pp = inverse of the UL factor of the nb x nb block at A (nb <= FACTOR_NB).
 template <typename T>
 inline int diag_ul_inv(const T *A, long long lda, T *U, long long ldu, int nb, long long col_base,
-                       cudaStream_t s) {
-    diag_ul_inv_kernel<T><<<1, DIAG_THREADS, 0, s>>>(A, lda, U, ldu, nb, col_base);
+                       cudaStream_t s, const int *skip = nullptr) {
+    constexpr int TG = DiagCfg<T>::TG;
+    diag_ul_inv_kernel<T><<<1, TG * TG, 0, s>>>(A, lda, U, ldu, nb, col_base, skip);
     return launch_status();
 }
 
@@ -422,8 +436,7 @@ inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, i
     // GPTQ_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
     static const bool blocked = tc::env_ll("GPTQ_LEAF", 1) != 0;
     if (!blocked) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
-    cudaFuncSetAttribute(leaf_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)LEAF_BLK_SMEM);
+    GPTQ_SMEM_LIMIT(leaf_blk_kernel, LEAF_BLK_SMEM);
     return launch_kernel(leaf_blk_kernel, dim3(1), dim3(LEAF_THREADS), LEAF_BLK_SMEM, s, pdl, A,
                          lda, U, ldu, nb, col_base);
 }
@@ -485,9 +498,7 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
     FactorStreams *fs = factor_streams(slot);
     if (!fs) return GPTQ_ERR_CUDA;
     std::lock_guard<std::mutex> lk(fs->mu);
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sm_count();
     // persistent CTAs of each side-stream GEMM: the rest of the SMs stay free for the chain
     static const long long side_env = tc::env_ll("GPTQ_FACTOR_SIDE_CTAS", 0);
     const int side = side_env > 0 ? (int)side_env : (2 * sms) / 3;

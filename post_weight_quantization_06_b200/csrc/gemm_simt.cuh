@@ -29,6 +29,7 @@ struct GemmArgs {
                         // that kernels on other streams keep SMs
     int pdl;            // SIMT path: launch as a programmatic dependent of the stream's previous
                         // kernel (the launch overlaps that kernel's tail)
+    const int *skip;    // when set and *skip != 0 the launch does nothing
 };
 
 namespace simt {
@@ -45,6 +46,7 @@ __global__ __launch_bounds__(256) void gemm_simt_kernel(GemmArgs<TA, TB> p) {
     const int i0 = blockIdx.y * BM, j0 = blockIdx.x * BN;
     if (p.c_upper && i0 >= j0 + BN) return;
     pdl_wait_prev();
+    if (p.skip && *p.skip) return;
     __shared__ __align__(16) float As[BK][BM + 4];
     __shared__ __align__(16) float Bs[BK][BN + 4];
     const int tid = threadIdx.x;
@@ -162,7 +164,7 @@ template <typename TA, typename TB>
 inline int gemm_simt(const GemmArgs<TA, TB> &p, cudaStream_t s) {
     if (p.M <= 0 || p.N <= 0) return GPTQ_OK;
     // fewer than ~one 128-tile wave: use 64 x 64 tiles for four times the CTAs
-    KtSpan span(s);
+    KtSpan span(s, p.skip != nullptr);
     int st;
     if ((long long)ceil_div(p.M, 128) * ceil_div(p.N, 128) < 148) {
         dim3 grid(ceil_div(p.N, 64), ceil_div(p.M, 64));
@@ -188,6 +190,7 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.c_upper = 0; p.a_upper = 0; p.b_upper = 0; p.a_lower = 0; p.b_lower = 0;
     p.max_ctas = 0;
     p.pdl = 0;
+    p.skip = nullptr;
     return p;
 }
 
@@ -205,6 +208,7 @@ struct F64Epilogue {
     double beta = 0.0;
     const float *diag = nullptr;
     int c_upper = 0;
+    const int *skip = nullptr;   // when set and *skip != 0 the launch does nothing
 };
 
 // C = alpha * op(A) op(B) (+ epilogue) accumulated in fp64 (64 x 64 tiles, 4 x 4 per thread).
@@ -224,6 +228,7 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
                                                           int b_upper, F64Epilogue ep,
                                                           double *part, int kchunk) {
     constexpr int T = F64_T, BK = F64_BK, PER = T * BK / 256;  // 8 elements per thread
+    if (ep.skip && *ep.skip) return;
     __shared__ double As[BK][T + 1];
     __shared__ double Bs[BK][T + 1];
     const int i0 = blockIdx.y * T, j0 = blockIdx.x * T;
@@ -304,11 +309,136 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
     }
 }
 
+// The same product for A not transposed and M >= 128: 128 x 64 tiles, 256 threads of 8 x 4
+// outputs each (a thread's 8 rows are contiguous, so its A values come as 16-byte shared loads
+// and every shared load feeds four fp64 FMAs), 16-deep K slabs double-buffered in shared memory
+// with the next slab's global loads in flight. B may be transposed; C may be upper (c_upper).
+constexpr int F64B_M = 128, F64B_N = 64, F64B_K = 16;
+
+template <typename TA, typename TB, typename TC>
+__global__ __launch_bounds__(256, 2) void gemm_f64acc_big_kernel(
+    int M, int N, int K, const TA *A, long long lda, const TB *B, long long ldb, int tb, TC *C,
+    long long ldc, double alpha, F64Epilogue ep, double *part, int kchunk) {
+    if (ep.skip && *ep.skip) return;
+    __shared__ __align__(16) double As[2][F64B_K][F64B_M];
+    __shared__ __align__(16) double Bs[2][F64B_K][F64B_N];
+    const int i0 = blockIdx.y * F64B_M, j0 = blockIdx.x * F64B_N;
+    if (ep.c_upper && i0 >= j0 + F64B_N) return;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int kbeg = blockIdx.z * kchunk, kend = min(K, kbeg + kchunk);
+    // A slab: row ar = tid / 2, k offsets 8 * (tid % 2) .. + 7
+    const int ar = tid >> 1, ak = (tid & 1) * 8;
+    // B slab (not transposed): k = tid / 16, columns 4 * (tid % 16) .. + 3;
+    // (transposed): column = tid / 4, k offsets 4 * (tid % 4) .. + 3
+    const int bk_n = tid >> 4, bn_n = (tid & 15) * 4;
+    const int bn_t = tid >> 2, bk_t = (tid & 3) * 4;
+    double ra[8], rb[4];
+    auto load = [&](int k0) {
+        const int gi = i0 + ar;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int gk = k0 + ak + e;
+            ra[e] = (gi < M && gk < kend) ? to_f64(A[(long long)gi * lda + gk]) : 0.0;
+        }
+        if (!tb) {
+            const int gk = k0 + bk_n;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int gj = j0 + bn_n + e;
+                rb[e] = (gj < N && gk < kend) ? to_f64(B[(long long)gk * ldb + gj]) : 0.0;
+            }
+        } else {
+            const int gj = j0 + bn_t;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int gk = k0 + bk_t + e;
+                rb[e] = (gj < N && gk < kend) ? to_f64(B[(long long)gj * ldb + gk]) : 0.0;
+            }
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) As[buf][ak + e][ar] = ra[e];
+        if (!tb) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) Bs[buf][bk_n][bn_n + e] = rb[e];
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) Bs[buf][bk_t + e][bn_t] = rb[e];
+        }
+    };
+    double acc[8][4];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    int buf = 0;
+    if (kbeg < kend) {
+        load(kbeg);
+        store(0);
+    }
+    __syncthreads();
+    for (int k0 = kbeg; k0 < kend; k0 += F64B_K) {
+        const bool more = k0 + F64B_K < kend;
+        if (more) load(k0 + F64B_K);   // in flight during the FMAs
+#pragma unroll
+        for (int kk = 0; kk < F64B_K; ++kk) {
+            double av[8], bv[4];
+            const double2 *ap = reinterpret_cast<const double2 *>(&As[buf][kk][ty * 8]);
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+                const double2 t = ap[h];
+                av[2 * h] = t.x;
+                av[2 * h + 1] = t.y;
+            }
+#pragma unroll
+            for (int b = 0; b < 4; ++b) bv[b] = Bs[buf][kk][tx + 16 * b];
+#pragma unroll
+            for (int a = 0; a < 8; ++a)
+#pragma unroll
+                for (int b = 0; b < 4; ++b) acc[a][b] = fma(av[a], bv[b], acc[a][b]);
+        }
+        if (more) store(buf ^ 1);
+        __syncthreads();
+        buf ^= 1;
+    }
+    if (part) {
+        double *P = part + (long long)blockIdx.z * M * N;
+#pragma unroll
+        for (int a = 0; a < 8; ++a) {
+            const int gi = i0 + ty * 8 + a;
+            if (gi >= M) continue;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int gj = j0 + tx + 16 * b;
+                if (gj < N) P[(long long)gi * N + gj] = acc[a][b];
+            }
+        }
+        return;
+    }
+    const double dg = ep.diag ? (double)*ep.diag : 0.0;
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const int gi = i0 + ty * 8 + a;
+        if (gi >= M) continue;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const int gj = j0 + tx + 16 * b;
+            if (gj >= N || (ep.c_upper && gj < gi)) continue;
+            double val = alpha * acc[a][b];
+            if (ep.Cin) val += ep.beta * (double)ep.Cin[(long long)gi * ep.ldcin + gj];
+            if (gi == gj) val += dg;
+            C[(long long)gi * ldc + gj] = (TC)val;
+        }
+    }
+}
+
 // C = alpha * sum_z part[z] (+ epilogue): the splits added in order, so the result does not
 // depend on scheduling.
 template <typename TC>
 __global__ void f64acc_reduce_kernel(int M, int N, int splits, const double *part, TC *C,
                                      long long ldc, double alpha, F64Epilogue ep) {
+    if (ep.skip && *ep.skip) return;
     const long long total = (long long)M * N;
     const double dg = ep.diag ? (double)*ep.diag : 0.0;
     for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
@@ -335,11 +465,37 @@ inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, 
                        long long ldb, int tb, TC *C, long long ldc, double alpha, cudaStream_t s,
                        int b_upper = 0, F64Epilogue ep = F64Epilogue(), F64Split sp = F64Split()) {
     if (M <= 0 || N <= 0) return GPTQ_OK;
+    const int sms = device_sm_count();
+    if (!ta && !b_upper && M >= F64B_M && N >= 32) {
+        // large products: 128 x 64 tiles, split K below two resident CTAs per SM
+        dim3 g2(ceil_div(N, F64B_N), ceil_div(M, F64B_M), 1);
+        const long long tiles = (long long)g2.x * g2.y;
+        int splits = 1;
+        if (sp.part && tiles < 2LL * sms && K >= 1024) {
+            splits = (int)((2LL * sms + tiles - 1) / tiles);
+            if (splits > K / 256) splits = K / 256;
+            if (splits > 16) splits = 16;
+            while (splits > 1 && (size_t)splits * M * N > sp.part_elems) --splits;
+        }
+        int kchunk = K;
+        if (splits > 1) {
+            kchunk = ceil_div(ceil_div(K, splits), F64B_K) * F64B_K;
+            splits = ceil_div(K, kchunk);
+        }
+        g2.z = splits;
+        gemm_f64acc_big_kernel<TA, TB, TC><<<g2, 256, 0, s>>>(
+            M, N, K, A, lda, B, ldb, tb, C, ldc, alpha, ep, splits > 1 ? sp.part : nullptr, kchunk);
+        if (int st = launch_status()) return st;
+        if (splits > 1) {
+            const long long total = (long long)M * N;
+            const int blocks = (int)((total + 255) / 256 < 4LL * sms ? (total + 255) / 256 : 4LL * sms);
+            f64acc_reduce_kernel<TC><<<blocks, 256, 0, s>>>(M, N, splits, sp.part, C, ldc, alpha, ep);
+            return launch_status();
+        }
+        return GPTQ_OK;
+    }
     dim3 grid(ceil_div(N, F64_T), ceil_div(M, F64_T), 1);
     // split K when the output tiles fill less than two waves and K is long
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long tiles = (long long)grid.x * grid.y;
     int splits = 1;
     if (sp.part && tiles < 2LL * sms && K >= 2048) {

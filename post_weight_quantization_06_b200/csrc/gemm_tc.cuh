@@ -139,6 +139,7 @@ struct TcGemmParams {
     long long wait_limit;
     int c_tma;          // 1: beta is 0 or 1 and cmap covers C; slices may leave by tensor store /
                         // tensor add-reduction instead of a read-modify-write
+    const int *skip;    // when set and *skip != 0 the launch does nothing
 };
 
 // Bulk tensor writes of one 32 x 32 slice from shared memory (128-byte swizzle) through the C
@@ -210,6 +211,7 @@ __device__ __forceinline__ void epi_load_c(const TcGemmParams &p, int row_base, 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                const __grid_constant__ CUtensorMap cmap, TcGemmParams p) {
+    if (p.skip && *p.skip) return;   // before any barrier, TMEM or copy: every thread leaves
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -537,9 +539,10 @@ namespace gptq {
 // GPTQ_FORCE_SIMT_GEMM is set).
 inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+    static const bool force_simt = std::getenv("GPTQ_FORCE_SIMT_GEMM") != nullptr;
     const bool small = (long long)g.M * g.N < 128LL * 256 || g.K < 64;
     if (small || !tcg::tc_eligible(g.A, g.lda, g.B, g.ldb) ||
-        (reinterpret_cast<uintptr_t>(g.C) & 3u) || std::getenv("GPTQ_FORCE_SIMT_GEMM"))
+        (reinterpret_cast<uintptr_t>(g.C) & 3u) || force_simt)
         return gemm_simt(g, s);
     tcg::TcGemmParams p;
     p.M = g.M; p.N = g.N; p.K = g.K;
@@ -552,6 +555,7 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     p.tiles_m = ceil_div(g.M, tcg::TILE);
     p.tiles_n = ceil_div(g.N, tcg::TILE);
     p.wait_limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
+    p.skip = g.skip;
     CUtensorMap am, bm, cm;
     const bool ok_a = p.a_mn ? tcg::make_map_f32(&am, g.A, g.K, g.M, g.lda, 32, 32, true)
                              : tcg::make_map_f32(&am, g.A, g.M, g.K, g.lda, 32, tcg::TILE, false);
@@ -564,15 +568,12 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
               (reinterpret_cast<uintptr_t>(g.C) & 15u) == 0 && g.ldc % 4 == 0 &&
               tcg::make_map_f32(&cm, g.C, g.M, g.N, g.ldc, 32, 32, false);
     if (!p.c_tma) cm = am;   // not read
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sm_count();
     const int tiles = tcg::num_tiles(p);
     int grid = tiles < sms ? tiles : sms;
     if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
-    cudaFuncSetAttribute(tcg::gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)tcg::SMEM_BYTES);
-    KtSpan span(s);
+    GPTQ_SMEM_LIMIT(tcg::gemm_tc_kernel, tcg::SMEM_BYTES);
+    KtSpan span(s, g.skip != nullptr);
     tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, cm, p);
     const int st = launch_status();
     span.done(KT_TC, g);

@@ -66,17 +66,20 @@ inline ILWork carve_ilwork(Carver &c, long long dim, int r) {
     const int p = il_block_p((int)dim, r);
     w.Y = c.take<float>((size_t)dim * p);
     w.Z = c.take<float>((size_t)dim * p);
-    w.Qsel = c.take<float>((size_t)p * r);
     w.HY = c.take<double>((size_t)dim * p);
     w.Tm = c.take<double>((size_t)p * p);
     w.ev = c.take<double>((size_t)p);
+    w.Qr = c.take<double>((size_t)p * r);
     w.G = c.take<double>((size_t)p * p);
     w.Gi = c.take<double>((size_t)p * p);
+    w.V64 = c.take<double>((size_t)dim * r);
     w.B12 = c.take<double>((size_t)dim * r);
     w.Y1 = c.take<double>((size_t)dim * r);
     w.Yr = c.take<float>((size_t)dim * r);
     w.C = c.take<double>((size_t)r * r);
     w.Ci = c.take<double>((size_t)r * r);
+    w.res = c.take<double>((size_t)r * ceil_div(dim, RES_ROWS) + 1);
+    w.ctl = c.take<int>(IL_CTL_WORDS);
     w.part_elems = (size_t)4 * dim * p;
     w.part = c.take<double>(w.part_elems);
     return w;
@@ -197,18 +200,50 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[GPTQ_NOALLOC_SC
 
 constexpr int kMaxDevices = 64;
 static void *g_noalloc_ptr[kMaxDevices];
+static unsigned long long g_noalloc_ctx[kMaxDevices];
 static std::mutex g_noalloc_mutex;
 
-// Device address of g_noalloc_scratch on the current device (looked up on the first call per
-// device), or nullptr if the lookup fails.
+// Unique id of the calling thread's current context (never reused within the process), or 0
+// when there is no current context or the driver does not provide the call.
+inline unsigned long long current_context_id() {
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_noalloc_scratch on the current device, or nullptr if the lookup fails.
+// The address belongs to the module loaded in one context: it is looked up on the first call
+// per device and again whenever that device's current context is not the one it was looked
+// up in (e.g. after cudaDeviceReset made the runtime create a new primary context).
 inline void *noalloc_scratch() {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
+    const unsigned long long ctx = current_context_id();
+    if (!g_noalloc_ptr[dev] || ctx == 0 || ctx != g_noalloc_ctx[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
         g_noalloc_ptr[dev] = p;
+        g_noalloc_ctx[dev] = current_context_id();   // the lookup made the context current
     }
     return g_noalloc_ptr[dev];
 }
@@ -258,6 +293,8 @@ GPTQ_API const char *gptq_status_string(int status) {
         case GPTQ_ERR_TIMEOUT: return "GPTQ_ERR_TIMEOUT: a bounded device wait gave up";
         case GPTQ_ERR_CUDA: return "GPTQ_ERR_CUDA: CUDA runtime error";
         case GPTQ_ERR_WORKSPACE: return "GPTQ_ERR_WORKSPACE: workspace missing, misaligned or too small";
+        case GPTQ_ERR_NOT_CONVERGED:
+            return "GPTQ_ERR_NOT_CONVERGED: the eigenvector iteration reached its cap before its residual test passed";
         default: return "unknown gptq status";
     }
 }
@@ -440,7 +477,7 @@ static int gptq_il_quantize_layer_body(const void *W, int w_dtype, int64_t m, in
         if (int st = prepare_hinv_impl(H, (int)n, lambda_rel, w.Uaug, n, lambda_out, w.f, s)) return st;
     } else {
         if (int st = il_top_eigvecs(H, n, (int)n, r, L, w.il, s)) return st;
-        if (int st = il_factor(H, n, (int)n, r, L, lambda_rel, w.Uaug, w.f.A, w.f.T, lambda_out,
+        if (int st = il_factor(H, n, (int)n, r, lambda_rel, w.Uaug, w.f.A, w.f.T, lambda_out,
                                w.il, s))
             return st;
     }

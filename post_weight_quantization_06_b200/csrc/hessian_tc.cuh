@@ -587,8 +587,7 @@ inline int hessian_tc(float *H, const __nv_bfloat16 *X, long long k, int n, cuda
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return GPTQ_ERR_CUDA;
-    cudaFuncSetAttribute(hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)SMEM_BYTES);
+    GPTQ_SMEM_LIMIT(hessian_tc_kernel, SMEM_BYTES);
     HessianParams p;
     p.H = H;
     p.n = n;
@@ -610,9 +609,7 @@ inline int hessian_tc(float *H, const __nv_bfloat16 *X, long long k, int n, cuda
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    int dev = 0, sms = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int sms = device_sm_count();
     cfg.gridDim = dim3(2 * (sms / 2));
     int clusters = 0;
     if (cudaOccupancyMaxActiveClusters(&clusters, hessian_tc_kernel, &cfg) != cudaSuccess ||

@@ -5,9 +5,10 @@
 // error and become R; the singular augmented Hessian is factored without a plain Cholesky.
 //
 // Device route:
-//   1. V_r: block subspace iteration on H (= 2 X^T X, same eigenvectors as X^T X) with
-//      CholeskyQR2 re-orthonormalisation, then a Rayleigh-Ritz step whose small p x p
-//      eigenproblem is solved by a one-CTA parallel-order Jacobi sweep.
+//   1. V_r: block subspace iteration on H (= 2 X^T X, same eigenvectors as X^T X): a few
+//      fp32-accurate tensor-core power steps, then fp64 iterations with CholeskyQR2
+//      re-orthonormalisation and a Rayleigh-Ritz step (eig.cuh) until every top-r Ritz pair
+//      passes a relative residual test (see il_top_eigvecs).
 //   2. H~ = [[H + l I, H V], [V^T H, V^T H V + l I]] with l = lambda_rel * mean of
 //      its n + r raw diagonal entries. The first n rows of U~ (H~^-1 = U~^T U~) are
 //      [U11, U12] with U11 the factor of the Schur complement S = H + l I - H V C^-1 V^T H
@@ -21,6 +22,7 @@
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "factor.cuh"
+#include "eig.cuh"
 
 namespace gptq {
 
@@ -51,122 +53,21 @@ __global__ void random_block_kernel(float *Y, long long total, unsigned long lon
     }
 }
 
-// One-CTA cyclic Jacobi on a symmetric p x p matrix (p even, p <= 128), round-robin
-// ordering so that p/2 disjoint rotations run at once. The matrix is held in fp64, the
-// accumulated rotations in fp32 (both in shared memory). On exit the r largest eigenvalues
-// are written in decreasing order to evals[0..r) and their eigenvectors to the columns of
-// Qsel (p x r).
-__global__ __launch_bounds__(512) void jacobi_eig_kernel(const double *Tin, int p, int r,
-                                                         float *Qsel, double *evals) {
-    extern __shared__ __align__(16) unsigned char jsm[];
-    const int LD = p + 1;
-    double *T = reinterpret_cast<double *>(jsm);
-    double *cs = T + p * LD;      // p/2 cosines
-    double *sn = cs + p / 2;      // p/2 sines
-    float *Q = reinterpret_cast<float *>(sn + p / 2);
-    int *pi = reinterpret_cast<int *>(Q + p * LD);
-    int *pj = pi + p / 2;
-    __shared__ double red[2];
-    const int tid = threadIdx.x, nt = blockDim.x;
-    const int warp = tid >> 5, lane = tid & 31, nwarps = nt >> 5;
-    for (int idx = tid; idx < p * p; idx += nt) {
-        const int i = idx / p, j = idx % p;
-        T[i * LD + j] = 0.5 * (Tin[i * p + j] + Tin[j * p + i]);
-        Q[i * LD + j] = (i == j) ? 1.f : 0.f;
-    }
-    const int half = p / 2;
-    for (int sweep = 0; sweep < 20; ++sweep) {
-        if (tid < 2) red[tid] = 0.0;
-        __syncthreads();
-        double off = 0.0, dia = 0.0;
-        for (int idx = tid; idx < p * p; idx += nt) {
-            const int i = idx / p, j = idx % p;
-            const double v = T[i * LD + j];
-            if (i != j) off += v * v; else dia += v * v;
-        }
-        off = warp_sum_d(off);
-        dia = warp_sum_d(dia);
-        if ((tid & 31) == 0) { atomicAdd(&red[0], off); atomicAdd(&red[1], dia); }
-        __syncthreads();
-        const bool done = red[0] <= 1e-26 * red[1];
-        __syncthreads();
-        if (done) break;
-        for (int rnd = 0; rnd < p - 1; ++rnd) {
-            for (int k = tid; k < half; k += nt) {
-                const int xb = p - 1 - k;
-                const int a = k == 0 ? 0 : 1 + (k - 1 + rnd) % (p - 1);
-                const int b = 1 + (xb - 1 + rnd) % (p - 1);
-                const int i = min(a, b), j = max(a, b);
-                pi[k] = i; pj[k] = j;
-                const double aij = T[i * LD + j];
-                double c = 1.0, sv = 0.0;
-                if (aij != 0.0) {
-                    const double tau = (T[j * LD + j] - T[i * LD + i]) / (2.0 * aij);
-                    const double t = (tau >= 0.0 ? 1.0 : -1.0) / (fabs(tau) + sqrt(1.0 + tau * tau));
-                    c = 1.0 / sqrt(1.0 + t * t);
-                    sv = t * c;
-                }
-                cs[k] = c; sn[k] = sv;
-            }
-            __syncthreads();
-            // rows i, j of every pair (warp per pair, lanes along the row), then the columns
-            for (int k = warp; k < half; k += nwarps) {
-                const int i = pi[k], j = pj[k];
-                const double c = cs[k], sv = sn[k];
-                for (int l = lane; l < p; l += 32) {
-                    const double ti = T[i * LD + l], tj = T[j * LD + l];
-                    T[i * LD + l] = c * ti - sv * tj;
-                    T[j * LD + l] = sv * ti + c * tj;
-                }
-            }
-            __syncthreads();
-            for (int k = warp; k < half; k += nwarps) {
-                const int i = pi[k], j = pj[k];
-                const double c = cs[k], sv = sn[k];
-                for (int l = lane; l < p; l += 32) {
-                    const double ti = T[l * LD + i], tj = T[l * LD + j];
-                    T[l * LD + i] = c * ti - sv * tj;
-                    T[l * LD + j] = sv * ti + c * tj;
-                    const float qi = Q[l * LD + i], qj = Q[l * LD + j];
-                    Q[l * LD + i] = (float)(c * qi - sv * qj);
-                    Q[l * LD + j] = (float)(sv * qi + c * qj);
-                }
-            }
-            __syncthreads();
-        }
-    }
-    for (int i = tid; i < p; i += nt) {
-        const double li = T[i * LD + i];
-        int rank = 0;
-        for (int j = 0; j < p; ++j) {
-            const double lj = T[j * LD + j];
-            rank += (lj > li) || (lj == li && j < i);
-        }
-        if (rank < r) {
-            evals[rank] = li;
-            for (int l = 0; l < p; ++l) Qsel[l * r + rank] = Q[l * LD + i];
-        }
-    }
-}
-
-inline size_t jacobi_smem(int p) {
-    return (size_t)p * (p + 1) * sizeof(double) + (size_t)p * sizeof(double) +
-           (size_t)p * (p + 1) * sizeof(float) + (size_t)p * sizeof(int);
-}
-
-// Columns of V (n x r): flip so that the largest-magnitude entry (first on ties) is positive.
-__global__ void sign_fix_kernel(float *V, int n, int r) {
+// Columns of V64 (n x r, fp64): flip so that the largest-magnitude entry (first on ties) is
+// positive; the same flip goes to the matching column of Qr (p x r), and V (fp32) receives the
+// rounded result.
+__global__ void sign_fix_kernel(double *V64, float *V, int n, int r, double *Qr, int p) {
     const int c = blockIdx.x;
-    __shared__ float bv[32];
+    __shared__ double bv[32];
     __shared__ int bi[32];
-    float best = -1.f;
+    double best = -1.0;
     int besti = 0;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const float a = fabsf(V[(long long)i * r + c]);
+        const double a = fabs(V64[(long long)i * r + c]);
         if (a > best) { best = a; besti = i; }
     }
     for (int o = 16; o > 0; o >>= 1) {
-        const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+        const double ob = __shfl_xor_sync(0xffffffffu, best, o);
         const int oi = __shfl_xor_sync(0xffffffffu, besti, o);
         if (ob > best || (ob == best && oi < besti)) { best = ob; besti = oi; }
     }
@@ -178,9 +79,13 @@ __global__ void sign_fix_kernel(float *V, int n, int r) {
         bi[0] = besti;
     }
     __syncthreads();
-    const bool flip = V[(long long)bi[0] * r + c] < 0.f;
-    if (flip)
-        for (int i = threadIdx.x; i < n; i += blockDim.x) V[(long long)i * r + c] = -V[(long long)i * r + c];
+    const double sg = V64[(long long)bi[0] * r + c] < 0.0 ? -1.0 : 1.0;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const double v = sg * V64[(long long)i * r + c];
+        V64[(long long)i * r + c] = v;
+        V[(long long)i * r + c] = (float)v;
+    }
+    for (int k = threadIdx.x; k < p; k += blockDim.x) Qr[(long long)k * r + c] *= sg;
 }
 
 // l~ = lambda_rel * (sum diag H + sum diag C) / (n + r); then C += l~ I.
@@ -207,82 +112,237 @@ __global__ void il_lambda_kernel(const float *H, long long ldh, int n, double *C
     for (int i = threadIdx.x; i < r; i += blockDim.x) C[i * r + i] += (double)l;
 }
 
+// Control words of the eigenvector iteration (device memory, see il_top_eigvecs): per phase a
+// done flag and a count of residual tests, and the residual kernel's CTA counter.
+enum {
+    IL_CTL_DONE = 0, IL_CTL_ITERS = 1,     // phase 2 (fp64)
+    IL_CTL_DONE1 = 2, IL_CTL_CHECKS1 = 3,  // phase 1 (fp32-accurate tensor-core products)
+    IL_CTL_COUNTER = 4, IL_CTL_WORDS = 8
+};
+
+// Relative residuals of the top r Ritz pairs, r_c = || H v_c - theta_c v_c || / theta_c with
+// v_c = Y Qr[:, c] and H v_c = HY Qr[:, c] (fp64 arithmetic). Each CTA sums r_c^2 over 32 rows
+// for 64 columns and writes its partial; the last CTA to finish adds the partials in a fixed
+// order and takes the decision of its phase:
+//   phase 2: done when max_c r_c <= tol;
+//   phase 1: done when max_c r_c <= tol or when it is above half the previous test's value
+//            (the fp32-accurate products have reached their floor);
+// it counts the test and stores max_c r_c in *resid. Nothing happens once the phase is done.
+constexpr int RES_ROWS = 32, RES_COLS = 64, RES_THREADS = 256;
+
+inline size_t il_residual_smem(int p) {
+    return sizeof(double) * ((size_t)p * RES_COLS + 2 * (size_t)RES_ROWS * p);
+}
+
+template <typename THY>
+__global__ __launch_bounds__(RES_THREADS) void il_residual_kernel(
+    const THY *HY, const float *Y, const double *Qr, const double *ev, int n, int p, int r,
+    double *part, int *ctl, int phase, double tol, double *resid) {
+    const int done_w = phase == 1 ? IL_CTL_DONE1 : IL_CTL_DONE;
+    const int count_w = phase == 1 ? IL_CTL_CHECKS1 : IL_CTL_ITERS;
+    if (ctl[done_w]) return;
+    extern __shared__ __align__(16) double rsm[];
+    double *Qc = rsm;                        // p x 64
+    double *HYs = Qc + p * RES_COLS;         // 32 x p
+    double *Ys = HYs + RES_ROWS * p;         // 32 x p
+    __shared__ double red[RES_THREADS / RES_COLS][RES_COLS];
+    __shared__ int last;
+    const int tid = threadIdx.x;
+    const int c0 = blockIdx.y * RES_COLS, i0 = blockIdx.x * RES_ROWS;
+    const int nc = min(RES_COLS, r - c0);
+    for (int idx = tid; idx < p * RES_COLS; idx += RES_THREADS) {
+        const int k = idx / RES_COLS, c = idx % RES_COLS;
+        Qc[idx] = c < nc ? Qr[(long long)k * r + c0 + c] : 0.0;
+    }
+    for (int idx = tid; idx < RES_ROWS * p; idx += RES_THREADS) {
+        const int i = idx / p, k = idx % p;
+        const long long row = i0 + i;
+        HYs[idx] = row < n ? (double)HY[row * p + k] : 0.0;
+        Ys[idx] = row < n ? (double)Y[row * p + k] : 0.0;
+    }
+    __syncthreads();
+    const int c = tid % RES_COLS, g = tid / RES_COLS;
+    const double th = c < nc ? ev[c0 + c] : 0.0;
+    double acc = 0.0;
+    for (int i = g; i < RES_ROWS; i += RES_THREADS / RES_COLS) {
+        double a = 0.0, b = 0.0;
+        for (int k = 0; k < p; ++k) {
+            const double q = Qc[k * RES_COLS + c];
+            a = fma(HYs[i * p + k], q, a);
+            b = fma(Ys[i * p + k], q, b);
+        }
+        const double rr = fma(-th, b, a);
+        acc = fma(rr, rr, acc);
+    }
+    red[g][c] = acc;
+    __syncthreads();
+    const int nblk = gridDim.x;
+    if (tid < nc) {
+        double t = 0.0;
+        for (int gg = 0; gg < RES_THREADS / RES_COLS; ++gg) t += red[gg][tid];
+        part[(long long)(c0 + tid) * nblk + blockIdx.x] = t;
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) last = atomicAdd(&ctl[IL_CTL_COUNTER], 1) == (int)(gridDim.x * gridDim.y) - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    double worst = 0.0;
+    const double floor = 1e-300 + 1e-14 * fabs(ev[0]);
+    for (int cc = tid; cc < r; cc += RES_THREADS) {
+        double t = 0.0;
+        for (int b = 0; b < nblk; ++b) t += *((volatile double *)&part[(long long)cc * nblk + b]);
+        worst = fmax(worst, sqrt(t) / fmax(fabs(ev[cc]), floor));
+    }
+    for (int o = 16; o > 0; o >>= 1) worst = fmax(worst, __shfl_xor_sync(0xffffffffu, worst, o));
+    __shared__ double wmax[RES_THREADS / 32];
+    if ((tid & 31) == 0) wmax[tid >> 5] = worst;
+    __syncthreads();
+    if (tid == 0) {
+        for (int w = 1; w < RES_THREADS / 32; ++w) worst = fmax(worst, wmax[w]);
+        const double prev = *resid;
+        const bool stalled = phase == 1 && ctl[count_w] > 0 && worst > 0.5 * prev;
+        *resid = worst;
+        ctl[count_w] += 1;
+        ctl[IL_CTL_COUNTER] = 0;
+        ctl[done_w] = (worst <= tol || stalled) ? 1 : 0;
+    }
+}
+
+// After the capped loop: GPTQ_ERR_NOT_CONVERGED (info = iterations run) if the residual test
+// never passed.
+__global__ void il_finish_kernel(const int *ctl) {
+    if (threadIdx.x == 0 && !ctl[IL_CTL_DONE]) report(GPTQ_ERR_NOT_CONVERGED, ctl[IL_CTL_ITERS]);
+}
+
 struct ILWork {
-    float *Y, *Z, *Qsel;       // subspace iteration blocks (n x p) and selected Ritz vectors
-    double *HY, *Tm, *ev;      // fp64 Rayleigh-Ritz: H Y (n x p), Y^T H Y (p x p), values
-    double *G, *Gi;            // p x p Gram and inverse UL factor
+    float *Y, *Z;              // n x p subspace blocks (fp32)
+    double *HY;                // n x p: H Y (fp64)
+    double *Tm, *ev, *Qr;      // Rayleigh-Ritz: Y^T H Y (p x p), Ritz values (p), vectors (p x r)
+    double *G, *Gi;            // p x p Gram and inverse UL factor (orthonormalisation)
+    double *V64;               // n x r Ritz vectors Y Qr
     double *B12, *Y1;          // n x r: H V and H V C^-1/2
     float *Yr;                 // n x r: H V C^-1
     double *C, *Ci;            // r x r extra block and inverse UL factor
+    double *res;               // residual partials (r x row blocks) and the last residual
+    int *ctl;                  // IL_CTL_WORDS control words
     double *part;              // split-K partial sums of the fp64-accumulating products
     size_t part_elems;         // 4 n p
 };
 
 inline F64Split il_split(const ILWork &w) { return F64Split{w.part, w.part_elems}; }
 
-constexpr int IL_ITERS_F32 = 4;   // power steps with fp32 accumulation
-constexpr int IL_ITERS_F64 = 1;   // then with fp64 accumulation, before Rayleigh-Ritz
+inline F64Epilogue skip_if(const int *flag) {
+    F64Epilogue ep;
+    ep.skip = flag;
+    return ep;
+}
+
+// Stopping rule of the eigenvector iteration: every one of the top r Ritz pairs has
+// || H v - theta v || <= IL_TOL * theta, with at most IL_MAX_ITERS fp64 iterations
+// (GPTQ_IL_MAX_ITERS overrides the cap, read at each call). Phase 1 runs at most
+// IL_P1_STEPS power steps with a residual test every IL_P1_EVERY steps.
+constexpr int IL_P1_STEPS = 24, IL_P1_EVERY = 4;
+constexpr double IL_P1_TOL = 1e-4;
+constexpr int IL_MAX_ITERS = 12;
+constexpr double IL_TOL = 5e-6;
 
 // dst = src Ubar^-T where src^T src = Ubar Ubar^T (Gram, factor and product in fp64):
 // dst has orthonormal columns spanning src.
-inline int cholqr_f64(const float *src, float *dst, int n, int p, ILWork &w, cudaStream_t s) {
-    if (int st = gemm_f64acc<float, float, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0,
+template <typename TS>
+inline int cholqr_f64(const TS *src, float *dst, int n, int p, ILWork &w, cudaStream_t s,
+                      const int *skip = nullptr) {
+    if (int st = gemm_f64acc<TS, TS, double>(p, p, n, src, p, 1, src, p, 0, w.G, p, 1.0,
+            s, 0, skip_if(skip), il_split(w))) return st;
+    if (int st = diag_ul_inv<double>(w.G, p, w.Gi, p, p, 0, s, skip)) return st;
+    return gemm_f64acc<TS, double, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.0,
+            s, 0, skip_if(skip), il_split(w));
+}
+
+// Top-r eigenvectors of the symmetric n x n matrix H: V (n x r, fp32, decreasing eigenvalue,
+// largest-magnitude entry of each column positive); also V64 (fp64) and B12 = H V64 in the
+// workspace. Subspace iteration on a block of p columns:
+//   phase 1: power steps Y <- orth(H Y) with fp32-accurate tensor-core products, until a
+//            residual test every IL_P1_EVERY steps passes IL_P1_TOL or stops improving;
+//   phase 2: up to the cap, each iteration (after the first) Y <- orth(HY) twice over
+//            (CholeskyQR2), then HY = H Y and T = Y^T HY with fp64 accumulation, the top r
+//            eigenpairs of T (sym_eig_top), and the residual test. Once it passes, a device
+//            flag makes every later launch of the loop return at once, so Y, HY and the
+//            Ritz pairs stay those of the converged iteration.
+inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V, ILWork &w,
+                          cudaStream_t s, bool want_b12 = true) {
+    KtStageScope stage(GPTQ_KT_IL);
+    const int p = il_block_p(n, r);
+    static const long long cap_env = tc::env_ll("GPTQ_IL_MAX_ITERS", 0);
+    const long long cap_now = tc::env_ll("GPTQ_IL_MAX_ITERS", cap_env);
+    const int cap = cap_now > 0 ? (int)std::min<long long>(cap_now, 64) : IL_MAX_ITERS;
+    const int *done = w.ctl + IL_CTL_DONE, *done1 = w.ctl + IL_CTL_DONE1;
+    if (cudaMemsetAsync(w.ctl, 0, sizeof(int) * IL_CTL_WORDS, s) != cudaSuccess) return GPTQ_ERR_CUDA;
+    random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
+    GPTQ_CHECK_LAUNCH();
+    const int nblk = ceil_div(n, RES_ROWS);
+    const dim3 rgrid(nblk, ceil_div(r, RES_COLS));
+    const size_t rsmem = il_residual_smem(p);
+    double *resid = w.res + (size_t)r * nblk;
+    GPTQ_SMEM_LIMIT(il_residual_kernel<float>, il_residual_smem(EIG_MAXP));
+    GPTQ_SMEM_LIMIT(il_residual_kernel<double>, il_residual_smem(EIG_MAXP));
+    // phase 1: Z = H Y on the tensor cores (fp32 accuracy), Y = orth(Z); every IL_P1_EVERY
+    // steps the Ritz pairs of Y (from Z) are tested first
+    for (int it = 0; it < IL_P1_STEPS; ++it) {
+        auto pz = gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f);
+        pz.skip = done1;
+        if (int st = gemm_f32(pz, s)) return st;
+        if (it > 0 && it % IL_P1_EVERY == 0) {
+            if (int st = gemm_f64acc<float, float, double>(p, p, n, w.Y, p, 1, w.Z, p, 0, w.Tm, p,
+                    1.0, s, 0, skip_if(done1), il_split(w))) return st;
+            if (int st = sym_eig_top(w.Tm, p, r, w.ev, w.Qr, done1, s)) return st;
+            il_residual_kernel<float><<<rgrid, RES_THREADS, rsmem, s>>>(
+                w.Z, w.Y, w.Qr, w.ev, n, p, r, w.res, w.ctl, 1, IL_P1_TOL, resid);
+            GPTQ_CHECK_LAUNCH();
+        }
+        if (int st = cholqr_f64<float>(w.Z, w.Y, n, p, w, s, done1)) return st;
+    }
+    // phase 2: fp64 products, a residual test every iteration
+    for (int it = 0; it < cap; ++it) {
+        if (it > 0) {
+            if (int st = cholqr_f64<double>(w.HY, w.Z, n, p, w, s, done)) return st;
+            if (int st = cholqr_f64<float>(w.Z, w.Y, n, p, w, s, done)) return st;
+        }
+        if (int st = gemm_f64acc<float, float, double>(n, p, n, H, ldh, 0, w.Y, p, 0, w.HY, p,
+                1.0, s, 0, skip_if(done), il_split(w))) return st;
+        if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p,
+                1.0, s, 0, skip_if(done), il_split(w))) return st;
+        if (int st = sym_eig_top(w.Tm, p, r, w.ev, w.Qr, done, s)) return st;
+        il_residual_kernel<double><<<rgrid, RES_THREADS, rsmem, s>>>(
+            w.HY, w.Y, w.Qr, w.ev, n, p, r, w.res, w.ctl, 2, IL_TOL, resid);
+        GPTQ_CHECK_LAUNCH();
+    }
+    il_finish_kernel<<<1, 32, 0, s>>>(w.ctl);
+    GPTQ_CHECK_LAUNCH();
+    // V64 = Y Qr, signs fixed (Qr's columns follow), V = fp32(V64); B12 = H V64 = HY Qr
+    if (int st = gemm_f64acc<float, double, double>(n, r, p, w.Y, p, 0, w.Qr, r, 0, w.V64, r, 1.0,
             s, 0, F64Epilogue(), il_split(w))) return st;
-    if (int st = diag_ul_inv<double>(w.G, p, w.Gi, p, p, 0, s)) return st;
-    return gemm_f64acc<float, double, float>(n, p, p, src, p, 0, w.Gi, p, 1, dst, p, 1.0,
+    sign_fix_kernel<<<r, 256, 0, s>>>(w.V64, V, n, r, w.Qr, p);
+    GPTQ_CHECK_LAUNCH();
+    if (!want_b12) return GPTQ_OK;
+    return gemm_f64acc<double, double, double>(n, r, p, w.HY, p, 0, w.Qr, r, 0, w.B12, r, 1.0,
             s, 0, F64Epilogue(), il_split(w));
 }
 
-// Top-r eigenvectors of H (n x n) into V (n x r).
-inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V, ILWork &w,
-                          cudaStream_t s) {
-    KtStageScope stage(GPTQ_KT_IL);
-    const int p = il_block_p(n, r);
-    random_block_kernel<<<256, 256, 0, s>>>(w.Y, (long long)n * p, 0x5eed0f11ull);
-    GPTQ_CHECK_LAUNCH();
-    for (int it = 0; it < IL_ITERS_F32 + IL_ITERS_F64; ++it) {
-        // Z = H Y, then CholeskyQR2: Y <- orth(Z)
-        if (it < IL_ITERS_F32) {
-            if (int st = gemm_simt(gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f), s)) return st;
-        } else {
-            if (int st = gemm_f64acc<float, float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.0,
-                    s, 0, F64Epilogue(), il_split(w))) return st;
-        }
-        if (int st = cholqr_f64(w.Z, w.Y, n, p, w, s)) return st;
-        if (int st = cholqr_f64(w.Y, w.Z, n, p, w, s)) return st;
-        std::swap(w.Y, w.Z);
-    }
-    // Rayleigh-Ritz in fp64: Tm = Y^T (H Y)
-    if (int st = gemm_f64acc<float, float, double>(n, p, n, H, ldh, 0, w.Y, p, 0, w.HY, p, 1.0,
-            s, 0, F64Epilogue(), il_split(w))) return st;
-    if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p, 1.0,
-            s, 0, F64Epilogue(), il_split(w))) return st;
-    const size_t smem = jacobi_smem(p);
-    cudaFuncSetAttribute(jacobi_eig_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    jacobi_eig_kernel<<<1, 512, smem, s>>>(w.Tm, p, r, w.Qsel, w.ev);
-    GPTQ_CHECK_LAUNCH();
-    // V = Y Qsel
-    if (int st = gemm_f64acc<float, float, float>(n, r, p, w.Y, p, 0, w.Qsel, r, 0, V, r, 1.0,
-            s, 0, F64Epilogue(), il_split(w))) return st;
-    sign_fix_kernel<<<r, 256, 0, s>>>(V, n, r);
-    return launch_status();
-}
-
-// First n rows of U~ into Uaug (n x (n + r), ldu = n + r), lambda~ into *lam.
+// First n rows of U~ into Uaug (n x (n + r), ldu = n + r), lambda~ into *lam, from the
+// eigenvector step's V64 and B12 = H V64 (both fp64; V, the fp32 output, is V64 rounded).
 // The Schur complement S = H + l I - H V C^-1 V^T H cancels the large eigenvalues of H along
-// V down to about l; it is formed with fp64 accumulation from the fp32 H and V, and only the
-// (well conditioned) result is rounded to fp32 for the factor.
+// V down to about l; it is formed with fp64 accumulation from the fp32 H, and only the (well
+// conditioned) result is rounded to fp32 for the factor.
 // Awork: n x n scratch, T: FACTOR_NB x n scratch.
-inline int il_factor(const float *H, long long ldh, int n, int r, const float *V,
-                     float lambda_rel, float *Uaug, float *Awork, float *T, float *lam,
-                     ILWork &w, cudaStream_t s) {
+inline int il_factor(const float *H, long long ldh, int n, int r, float lambda_rel, float *Uaug,
+                     float *Awork, float *T, float *lam, ILWork &w, cudaStream_t s) {
     KtStageScope stage(GPTQ_KT_IL);
     const long long ldu = n + r;
-    // B12 = H V (n x r), C = V^T B12 (r x r)
-    if (int st = gemm_f64acc<float, float, double>(n, r, n, H, ldh, 0, V, r, 0, w.B12, r, 1.0,
-            s, 0, F64Epilogue(), il_split(w))) return st;
-    if (int st = gemm_f64acc<float, double, double>(r, r, n, V, r, 1, w.B12, r, 0, w.C, r, 1.0,
-            s, 0, F64Epilogue(), il_split(w))) return st;
+    // C = V64^T B12 (r x r)
+    if (int st = gemm_f64acc<double, double, double>(r, r, n, w.V64, r, 1, w.B12, r, 0, w.C, r,
+            1.0, s, 0, F64Epilogue(), il_split(w))) return st;
     il_lambda_kernel<<<1, 1024, 0, s>>>(H, ldh, n, w.C, r, lambda_rel, lam);
     GPTQ_CHECK_LAUNCH();
     // C = Ubar Ubar^T, Ci = Ubar^-1, C^-1 = Ci^T Ci
@@ -297,12 +357,13 @@ inline int il_factor(const float *H, long long ldh, int n, int r, const float *V
     ep.Cin = H; ep.ldcin = ldh; ep.beta = 1.0; ep.diag = lam; ep.c_upper = 1;
     if (int st = gemm_f64acc<double, double, float>(n, n, r, w.Y1, r, 0, w.Y1, r, 1, Awork, n, -1.0,
             s, 0, ep, il_split(w))) return st;
-    cudaMemsetAsync(Uaug, 0, sizeof(float) * (size_t)n * ldu, s);
+    if (cudaMemsetAsync(Uaug, 0, sizeof(float) * (size_t)n * ldu, s) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
     if (int st = factor_ul_inverse(Awork, n, Uaug, ldu, n, T, s)) return st;
     // U12 = -U11 Yr
-    auto p = gemm_args<float, float>(n, r, n, Uaug, ldu, 0, w.Yr, r, 0, Uaug + n, ldu, -1.f, 0.f);
-    p.a_upper = 1;
-    return gemm_f32(p, s);
+    auto pa = gemm_args<float, float>(n, r, n, Uaug, ldu, 0, w.Yr, r, 0, Uaug + n, ldu, -1.f, 0.f);
+    pa.a_upper = 1;
+    return gemm_f32(pa, s);
 }
 
 }  // namespace gptq

@@ -112,12 +112,14 @@ inline void kt_count(const GemmArgs<TA, TB> &g, double &flops, double &bytes) {
             c_elems * sizeof(float) * (g.beta != 0.f ? 2.0 : 1.0);
 }
 
-// Brackets one launch on stream s; inert unless the flag is set.
+// Brackets one launch on stream s; inert unless the flag is set, and for a conditional launch
+// (one that a device flag may turn into a no-op, whose work is therefore not known here).
 struct KtSpan {
     bool on;
     cudaStream_t s;
     cudaEvent_t a = nullptr, b = nullptr;
-    explicit KtSpan(cudaStream_t st) : on(kt_enabled()), s(st) {
+    explicit KtSpan(cudaStream_t st, bool conditional = false)
+        : on(kt_enabled() && !conditional), s(st) {
         if (!on) return;
         if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess ||
             cudaEventRecord(a, s) != cudaSuccess) {

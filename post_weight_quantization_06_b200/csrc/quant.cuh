@@ -265,8 +265,7 @@ inline size_t colloop_smem() {
 template <int NSLOT>
 inline int colloop_launch(const ColloopArgs &a, cudaStream_t s) {
     const size_t smem = colloop_smem<NSLOT>();
-    cudaFuncSetAttribute(colloop_kernel<NSLOT, COLLOOP_ROWS>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    GPTQ_SMEM_LIMIT((colloop_kernel<NSLOT, COLLOOP_ROWS>), smem);
     const int rows_per_cta = (COLLOOP_THREADS / 32) * COLLOOP_ROWS;
     colloop_kernel<NSLOT, COLLOOP_ROWS>
         <<<ceil_div(a.m, rows_per_cta), COLLOOP_THREADS, smem, s>>>(a);

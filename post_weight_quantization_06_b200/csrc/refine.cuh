@@ -236,8 +236,7 @@ inline int bidup_pass(const float *H, int m, int n, int bits, int gs, const floa
                       RefineWs &w, cudaStream_t s) {
     constexpr int B = BIDUP_B;
     const size_t smem = sizeof(float) * (B * B + B);
-    cudaFuncSetAttribute(bidup_block_kernel<B / 32, BIDUP_ROWS>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    GPTQ_SMEM_LIMIT((bidup_block_kernel<B / 32, BIDUP_ROWS>), smem);
     const int G = n / gs;
     const int rows_per_cta = (BIDUP_THREADS / 32) * BIDUP_ROWS;
     for (int j0 = 0; j0 < n; j0 += B) {
@@ -282,7 +281,7 @@ inline int il_refine(const TW *W, int m, int n, const float *H, int r, int bits,
                                                           1.f, 0.f), s)) return st;
             if (int st = gemm_f32(gemm_args<float, float>(m, m, n, w.Gm, n, 0, w.E, n, 1, w.Bm, m,
                                                           1.f, 0.f), s)) return st;
-            if (int st = il_top_eigvecs(w.Bm, m, m, r, w.P, w.il, s)) return st;
+            if (int st = il_top_eigvecs(w.Bm, m, m, r, w.P, w.il, s, false)) return st;
             if (int st = gemm_f32(gemm_args<float, float>(n, r, m, w.E, n, 1, w.P, r, 0, L, r,
                                                           1.f, 0.f), s)) return st;
             refine_transpose_kernel<<<blocks, 256, 0, s>>>(w.P, m, r, R);

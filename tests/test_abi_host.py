@@ -47,8 +47,9 @@ def test_library_has_no_dynamic_cuda_runtime_dependency():
 def test_status_strings():
     import post_weight_quantization_06_b200 as g
     assert g.status_string(0) == "GPTQ_OK"
-    for code in range(-6, 0):
+    for code in range(-7, 0):
         assert g.status_string(code).startswith("GPTQ_ERR_")
+    assert "NOT_CONVERGED" in g.status_string(g.GPTQ_ERR_NOT_CONVERGED)
     assert "unknown" in g.status_string(7)
 
 

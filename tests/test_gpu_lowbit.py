@@ -30,9 +30,11 @@ def _judge(label, q, codes_gpu, scales_gpu, zeros_gpu):
     assert agree >= CODE_AGREE and worst < CODE_BAND and srel <= 1e-6
 
 
+# the calibration's signal has rank r: beyond it the spectrum is a flat noise bulk whose
+# eigenvectors the pass cannot resolve (it reports GPTQ_ERR_NOT_CONVERGED there)
 @pytest.mark.parametrize("r,gsL", [(16, 128), (16, 0), (32, 64)])
 def test_lowrank_factors_at_4_and_8_bits(g, r, gsL):
-    L = datagen.lowrank(device=DEV, scale=0.0625, r=16)
+    L = datagen.lowrank(device=DEV, scale=0.0625, r=r)
     n, m = L.n, L.m
     H = torch.zeros(n, n, device=DEV)
     g.gptq_hessian_accumulate(H, L.X)

@@ -118,3 +118,23 @@ def test_residual_error_bound():
     Xt = np.hstack([X, X @ res["L"]])
     dl = ((Xt @ D.T) ** 2).sum(0)
     assert np.all(dl <= res["loss_rows"] / 2 * (1 + 1e-9))
+
+
+@pytest.mark.parametrize("seed,r,lam_rel", [(11, 3, 1e-3), (12, 6, 1e-4), (13, 0, 1e-2)])
+def test_il_damping_closed_form(seed, r, lam_rel):
+    """The relative damping of the augmented Hessian (config: lambda~ = lambda_rel * mean of
+    the diagonal of H~_raw = 2 X~^T X~ over all n + r coordinates). The extra columns X V_r
+    have squared norms sigma_i^2 (diag(V_r^T G V_r) = sigma^2 for exact eigenvectors), so
+    lambda~ = lambda_rel * 2 (||X||_F^2 + sum_{i<=r} sigma_i^2) / (n + r), with sigma taken
+    here from an SVD of X. A mean over n entries, or over X~^T X~ instead of 2 X~^T X~,
+    misses this value."""
+    n = 30
+    W, X = _lowrank_layer(seed, 3, n, 250, max(r, 1))
+    G = X.T @ X
+    V, _ = oracle.top_singular_directions(G, r)
+    _, lam = oracle.il_hessian(G, V, lam_rel)
+    sv = np.linalg.svd(X, compute_uv=False)
+    closed = lam_rel * 2.0 * ((X ** 2).sum() + (sv[:r] ** 2).sum()) / (n + r)
+    assert lam == pytest.approx(closed, rel=1e-12)
+    if r:
+        assert abs(lam - lam_rel * 2.0 * ((X ** 2).sum() + (sv[:r] ** 2).sum()) / n) > 1e-6 * lam

@@ -5,7 +5,8 @@ library's fixed device array instead of a workspace. This file is collected last
 
 The test calls it twice in a row through the C ABI and compares both results with the
 workspace entry point (same kernels, same inputs: the results must be identical, which is
-tighter than the parity tolerance), and checks the size limit."""
+tighter than the parity tolerance), checks that the second (warm) call changes neither torch's
+allocated bytes nor the device's free memory, and checks the size limit."""
 import ctypes
 
 import numpy as np
@@ -40,12 +41,18 @@ def test_noalloc_matches_workspace_entry_twice(wl, scale):
     g.gptq_quantize_layer(L.W, U, L.bits, L.group_size, L.block_size, *ref,
                           g.workspace(g.GPTQ_OP_QUANTIZE, m, n, 0, L.block_size))
     g.gptq_sync_status()
-    for _ in range(2):
+    for call in range(2):
         out = _outputs(m, n, L.bits, L.group_size)
+        torch.cuda.synchronize()
+        held, free = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         g.gptq_quantize_layer_noalloc(L.W, U, L.bits, L.group_size, L.block_size, *out)
         g.gptq_sync_status()
         for a, b in zip(ref, out):
             assert torch.equal(a, b)
+        if call == 1:
+            # the warm call takes no device memory: neither through torch nor from the driver
+            assert torch.cuda.memory_allocated() == held
+            assert torch.cuda.mem_get_info()[0] == free
 
 
 def test_noalloc_rejects_layers_beyond_the_scratch():

@@ -60,6 +60,8 @@ def parse_args(argv=None):
                     help="use only the first TOKENS calibration rows (small profiling cases)")
     ap.add_argument("--no-il", action="store_true",
                     help="skip the intrinsic-LoRA layer pass reported under 'il'")
+    ap.add_argument("--no-reduced", action="store_true",
+                    help="skip GPTQ with lattice basis reduction reported under 'reduced'")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads (tiny, attn, DeiT fc1/fc2) reported under 'configs'")
     return ap.parse_args(argv)
@@ -542,6 +544,59 @@ def run_other_workloads(g, dev, steps: int, warmup: int, rank: int) -> dict:
     return out
 
 
+def run_reduced(g, dev, steps: int, rank: int) -> dict:
+    """GPTQ with lattice basis reduction (gptq_quantize_layer_reduced) on the DeiT fc1 layer
+    (2-bit, per channel) and the tiny layer (4-bit, per channel): the whole entry point (LLL, the
+    rounding in the reduced basis, codes and loss) timed with CUDA events after one warm-up call,
+    with the LLL statistics and the loss against plain GPTQ on the same per-channel grid."""
+    import datagen
+    out = {}
+    for name, bits in (("deit_fc1", 2), ("tiny", 4)):
+        layer = datagen.WORKLOADS[name](device=dev, seed=rank_seed(name, rank))
+        m, n = layer.m, layer.n
+        s = torch.cuda.Stream(device=dev)
+        H = torch.zeros(n, n, device=dev)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(s):
+            g.gptq_hessian_accumulate(H, layer.X, stream=s)
+        res = dict(codes=torch.empty(m, n * bits // 32, dtype=torch.int32, device=dev),
+                   scales=torch.empty(m, device=dev),
+                   zeros=torch.empty(m, dtype=torch.uint8, device=dev),
+                   loss=torch.empty(m, dtype=torch.float64, device=dev),
+                   stats=torch.zeros(8, dtype=torch.int64, device=dev))
+        ws = g.workspace(g.GPTQ_OP_REDUCED, m, n, 0, 0, dev)
+
+        def call():
+            g.gptq_quantize_layer_reduced(layer.W, H, bits, layer.lambda_rel, res["codes"],
+                                          res["scales"], res["zeros"], res["loss"], None,
+                                          res["stats"], ws, stream=s)
+
+        with torch.cuda.stream(s):
+            call()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(s)
+            for _ in range(max(1, steps)):
+                call()
+            e1.record(s)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / max(1, steps)
+        st, _ = g.gptq_sync_status(s, raise_on_error=False)
+        # plain GPTQ on a per-channel grid, same bits and damping
+        plain = g.quantize_layer(layer.W, H=H, bits=bits, group_size=0,
+                                 lambda_rel=layer.lambda_rel, check_status=False)
+        torch.cuda.synchronize(dev)
+        stats = res["stats"].cpu().tolist()
+        out[name] = {"workload": f"{layer.name.split(',')[0]}, {layer.k} tokens, {bits}-bit per-channel",
+                     "ms": ms,
+                     "lll_swaps": stats[0], "lll_size_reductions": stats[1],
+                     "max_abs_T": stats[3], "codes_clipped": stats[4], "codes": m * n,
+                     "loss_vs_plain": float(res["loss"].sum().item() / plain["loss"].sum().item()),
+                     "device_status": int(st)}
+        del layer, H, res, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(layer, budget_s: float):
     """The fp64 oracle as it stands, on a bounded sample of the same layer, on the host cores:
     Hessian over a slice of the tokens, the full n x n factor, the sweep over a few rows;
@@ -664,6 +719,7 @@ def bench_ours(args):
     # the other workloads, each timed on its own after the main line's measurements
     other = None
     il = None
+    reduced = None
     if not args.no_configs or not args.no_il:
         del lp
         torch.cuda.empty_cache()
@@ -675,6 +731,8 @@ def bench_ours(args):
             torch.cuda.empty_cache()
         if not args.no_configs:
             other = run_other_workloads(g, dev, max(1, args.steps), max(1, min(args.warmup, 3)), rank)
+    if not args.no_reduced:
+        reduced = run_reduced(g, dev, 2, rank)
 
     if rank == 0:
         out = {
@@ -714,6 +772,8 @@ def bench_ours(args):
             out["il"] = il
         if other:
             out["configs"] = other
+        if reduced:
+            out["reduced"] = reduced
         if not args.no_cpu_baseline and world == 1:
             out["cpu_baseline"] = cpu_baseline(layer, args.cpu_budget_s)
         print(json.dumps(out))

@@ -11,6 +11,7 @@
  *   gptq_il_refine            OLrC + Bid-Up refinement rounds on a quantized layer: new L, R, codes
  *   gptq_quantize_lowrank     L and R stored at low precision (4-bit L, 8-bit R) on min-max grids
  *   gptq_2d_round             two-sided adaptive rounding of a real matrix to integers (GPTQ-2D)
+ *   gptq_quantize_layer_reduced  GPTQ after LLL reduction of the data lattice (per-channel grid)
  *   gptq_set_flags            synchronous status returns and debug synchronisation (see below)
  *   gptq_kernel_times         device time and algorithmic work of the GEMM launches (diagnostic)
  *
@@ -71,7 +72,8 @@ typedef enum {
     GPTQ_OP_QUANTIZE = 2,
     GPTQ_OP_IL_QUANTIZE = 3,
     GPTQ_OP_IL_REFINE = 4,
-    GPTQ_OP_2D_ROUND = 5
+    GPTQ_OP_2D_ROUND = 5,
+    GPTQ_OP_REDUCED = 6
 } gptq_op;
 
 /* Process-wide behaviour flags (gptq_set_flags; default 0):
@@ -372,6 +374,41 @@ GPTQ_API int gptq_quantize_lowrank(const float *L, const float *R, int64_t n, in
 GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G, const float *H,
                            int32_t *Z, float *err, void *workspace, size_t ws_bytes,
                            gptq_stream_t stream);
+
+/*
+ * gptq_quantize_layer_reduced — GPTQ with lattice basis reduction (WITHREDUCTION).
+ * The Lattice Geometry of Neural Network Quantization, section 5.2: reduce the basis of the
+ * regularised data lattice X' = [X; mu I] (mu^2 = lambda / 2) with LLL before running GPTQ /
+ * Babai on it, and map the integer coefficients back through the unimodular change of basis
+ * T. The page gives no procedure for the quantization grid; here it is per channel (one min-max
+ * scale and zero-point per output row, from the original row: every row's lattice is then s X',
+ * so one reduction serves the layer). Steps:
+ *   lambda = lambda_rel * mean(diag H); G' = (H + lambda I) / 2 (H's upper triangle read);
+ *   LLL (delta = 3/4, fp64, on the Gram matrix) of the column-reversed basis, reversed back:
+ *     GPTQ's natural column order is Babai's nearest plane on the reversed basis;
+ *   per row: s, z by the min-max rule; u = w / s + z; c' = one-sided adaptive rounding of
+ *     T^-1 u under G_red = T^T G' T (rint, ties to even, no clipping);
+ *   c = clip(T c', 0, maxq); codes packed as gptq_quantize_layer packs them.
+ *   W          device, m x n, w_dtype GPTQ_BF16 or GPTQ_F32; 1 <= m <= 65536.
+ *   H          device, n x n fp32 raw Hessian 2 X^T X; 1 <= n <= 2048.
+ *   bits       2..8 with n * bits % 32 == 0.
+ *   codes      device, m x (n * bits / 32) uint32.  scales, zeros: device, m fp32 / m uint8.
+ *   loss_out   device, m fp64 or NULL: (w - w_hat)^T (H + lambda I) (w - w_hat) per row.
+ *   coef_out   device, m x n int32 or NULL: the coefficients c' in the reduced basis.
+ *   stats_out  device, 8 int64 or NULL: [0] LLL swaps, [1] size reductions, [2] LLL loop
+ *              iterations, [3] largest |entry| of T and T^-1, [4] codes that clipping changed,
+ *              [5..7] zero.
+ *   workspace  device, >= gptq_workspace_size(GPTQ_OP_REDUCED, m, n, 0, 0) bytes.
+ * Argument errors: GPTQ_ERR_ARG, GPTQ_ERR_WORKSPACE (nothing enqueued). Device errors:
+ * GPTQ_ERR_NOT_PD (G' not numerically positive definite), GPTQ_ERR_NONFINITE (a weight),
+ * GPTQ_ERR_NOT_CONVERGED (the LLL loop passed its bound of 64 n^2 + 4096 iterations, info = swaps;
+ * or an entry of T beyond 2^24, info = -1).
+ */
+GPTQ_API int gptq_quantize_layer_reduced(const void *W, int w_dtype, int64_t m, int64_t n,
+                                         const float *H, int bits, float lambda_rel,
+                                         uint32_t *codes, float *scales, uint8_t *zeros,
+                                         double *loss_out, int32_t *coef_out, int64_t *stats_out,
+                                         void *workspace, size_t ws_bytes, gptq_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -43,6 +43,16 @@ gptq2d_* (two-sided rounding)   anti-diagonal sweep equals the vectorised sweep 
 gptq2d_residuals                closed form X - Z = U_G^T E U_H: equals the sweep's
                                 recorded v - z; every |c| <= 1/2 for the sweep's Z
                                 and a Z moved by one step breaks it
+lll_gram / reduce_for_gptq      the output is size-reduced and meets the Lovasz
+(lattice basis reduction)       condition (Gram-Schmidt data from an independent
+                                Cholesky), T is unimodular and G_red = T^T G T; the
+                                LLL bound |b_1|^2 <= 2^(n-1) lambda_1^2 against brute-
+                                force shortest vectors; a diagonal Gram is only
+                                permuted
+round_in_basis / withreduction  equals a data-space nearest plane on an explicit
+                                basis; orthogonal data gives round-to-nearest;
+                                Babai's bound sum Bn / 4 in the reduced basis; never
+                                better than the brute-force optimum on tiny rows
 ==============================  ==================================================
 """
 from .gptq import (
@@ -71,6 +81,7 @@ from .pack import pack_codes, unpack_codes
 from .refine import olrc, bidup, dequant, refine as refine_loop
 from .refine import data_loss_rows as lowrank_loss_rows
 from .lowbit import rtn_quantize, quantize_lowrank
+from .lll import lll_gram, gram_schmidt, reduce_for_gptq, round_in_basis, withreduction
 from .gptq2d import (adaptive_round_1d, gptq2d_antidiagonal, gptq2d_residuals, gptq2d_vectorized,
                      reverse_cholesky_upper, two_sided_loss)
 

@@ -20,7 +20,7 @@ GPTQ_ERR_TIMEOUT, GPTQ_ERR_CUDA, GPTQ_ERR_WORKSPACE = -4, -5, -6
 GPTQ_ERR_NOT_CONVERGED = -7
 GPTQ_BF16, GPTQ_F32 = 0, 1
 GPTQ_OP_HESSIAN, GPTQ_OP_PREPARE_HINV, GPTQ_OP_QUANTIZE, GPTQ_OP_IL_QUANTIZE = 0, 1, 2, 3
-GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND = 4, 5
+GPTQ_OP_IL_REFINE, GPTQ_OP_2D_ROUND, GPTQ_OP_REDUCED = 4, 5, 6
 GPTQ_FLAG_SYNC_STATUS, GPTQ_FLAG_DEBUG_CHECKS, GPTQ_FLAG_IL_FP64 = 1, 2, 4
 GPTQ_FLAG_KERNEL_TIMES = 8
 KT_STAGES = ("other", "factor", "sweep", "il", "refine", "2d")   # gptq_kt_stage order
@@ -31,7 +31,7 @@ EXPORTED = ("gptq_workspace_size", "gptq_status_string", "gptq_sync_status", "gp
             "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
             "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
             "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags",
-            "gptq_kernel_times")
+            "gptq_kernel_times", "gptq_quantize_layer_reduced")
 
 
 class KernelTime(ctypes.Structure):
@@ -74,6 +74,8 @@ def _load() -> ctypes.CDLL:
         "gptq_set_flags": (None, [ctypes.c_uint]),
         "gptq_get_flags": (ctypes.c_uint, []),
         "gptq_kernel_times": (c_int, [ctypes.POINTER(KernelTime), c_int]),
+        "gptq_quantize_layer_reduced": (c_int, [c_p, c_int, c_i64, c_i64, c_p, c_int, c_f, c_p, c_p,
+                                                c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -300,6 +302,48 @@ def gptq_2d_round(X: torch.Tensor, G: torch.Tensor, H: torch.Tensor, Z: torch.Te
     nbytes = 0 if ws is None else ws.numel()
     _check(_lib.gptq_2d_round(_ptr(X), m, n, _ptr(G), _ptr(H), _ptr(Z), _ptr(err), _ptr(ws),
                               nbytes, _stream(stream)), "gptq_2d_round")
+
+
+def gptq_quantize_layer_reduced(W: torch.Tensor, H: torch.Tensor, bits: int, lambda_rel: float,
+                                codes: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                                loss_out: torch.Tensor | None, coef_out: torch.Tensor | None,
+                                stats_out: torch.Tensor | None, ws: torch.Tensor, stream=None):
+    _dev(W, "W")
+    _dev(H, "H", torch.float32)
+    _dev(codes, "codes", torch.int32)
+    _dev(scales, "scales", torch.float32)
+    _dev(zeros, "zeros", torch.uint8)
+    if loss_out is not None:
+        _dev(loss_out, "loss_out", torch.float64)
+    if coef_out is not None:
+        _dev(coef_out, "coef_out", torch.int32)
+    if stats_out is not None:
+        _dev(stats_out, "stats_out", torch.int64)
+    m, n = W.shape
+    _check(_lib.gptq_quantize_layer_reduced(_ptr(W), _dtype_code(W), m, n, _ptr(H), bits,
+                                            float(lambda_rel), _ptr(codes), _ptr(scales),
+                                            _ptr(zeros), _ptr(loss_out), _ptr(coef_out),
+                                            _ptr(stats_out), _ptr(ws), ws.numel(), _stream(stream)),
+           "gptq_quantize_layer_reduced")
+
+
+def quantize_layer_reduced(W: torch.Tensor, H: torch.Tensor, *, bits: int, lambda_rel: float = 0.01,
+                           check_status: bool = True) -> dict:
+    """GPTQ after LLL reduction of the data lattice, per-channel grid, with fresh outputs."""
+    dev = W.device
+    m, n = W.shape
+    out = dict(codes=torch.empty(m, n * bits // 32, dtype=torch.int32, device=dev),
+               scales=torch.empty(m, dtype=torch.float32, device=dev),
+               zeros=torch.empty(m, dtype=torch.uint8, device=dev),
+               loss=torch.empty(m, dtype=torch.float64, device=dev),
+               coef=torch.empty(m, n, dtype=torch.int32, device=dev),
+               stats=torch.zeros(8, dtype=torch.int64, device=dev))
+    ws = workspace(GPTQ_OP_REDUCED, m, n, 0, 0, dev)
+    gptq_quantize_layer_reduced(W, H, bits, lambda_rel, out["codes"], out["scales"], out["zeros"],
+                                out["loss"], out["coef"], out["stats"], ws)
+    if check_status:
+        gptq_sync_status()
+    return out
 
 
 def round_2d(X: torch.Tensor, G: torch.Tensor, H: torch.Tensor, *, with_err: bool = False,

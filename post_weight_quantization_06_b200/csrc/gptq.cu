@@ -12,6 +12,7 @@
 #include "refine.cuh"
 #include "gptq2d.cuh"
 #include "hessian_tc.cuh"
+#include "lll.cuh"
 
 namespace gptq {
 
@@ -120,6 +121,40 @@ inline TwoDWs carve_2d(Carver &c, long long m, long long n) {
     w.E = c.take<float>((size_t)(w.Mp * w.Np));
     w.F = c.take<float>((size_t)(w.Mp * w.Np));
     w.lam = c.take<float>(2);
+    return w;
+}
+
+// Buffers of gptq_quantize_layer_reduced.
+struct ReducedWs {
+    float *lam, *Gd, *A2, *Gred, *Tf, *Tif, *U, *Up, *Cr, *D, *DH;
+    double *A, *Bn, *T, *Ti;
+    int32_t *Zi;
+    uint8_t *c8;
+    long long *stats;
+    TwoDWs w2;
+};
+constexpr int REDUCED_STATS = 8;
+inline ReducedWs carve_reduced(Carver &c, long long m, long long n) {
+    ReducedWs w;
+    w.stats = c.take<long long>(REDUCED_STATS);
+    w.lam = c.take<float>(2);
+    w.A = c.take<double>((size_t)n * n);
+    w.Bn = c.take<double>((size_t)n);
+    w.T = c.take<double>((size_t)n * n);
+    w.Ti = c.take<double>((size_t)n * n);
+    w.Gd = c.take<float>((size_t)n * n);
+    w.A2 = c.take<float>((size_t)n * n);
+    w.Gred = c.take<float>((size_t)n * n);
+    w.Tf = c.take<float>((size_t)n * n);
+    w.Tif = c.take<float>((size_t)n * n);
+    w.U = c.take<float>((size_t)m * n);
+    w.Up = c.take<float>((size_t)m * n);
+    w.Cr = c.take<float>((size_t)m * n);
+    w.D = c.take<float>((size_t)m * n);
+    w.DH = c.take<float>((size_t)m * n);
+    w.Zi = c.take<int32_t>((size_t)m * n);
+    w.c8 = c.take<uint8_t>((size_t)m * n);
+    w.w2 = carve_2d(c, m, n);
     return w;
 }
 
@@ -278,6 +313,10 @@ GPTQ_API size_t gptq_workspace_size(int op, int64_t m, int64_t n, int r, int blo
         case GPTQ_OP_2D_ROUND:
             if (m < 1 || m > 65536 || n > 65536) return 0;
             carve_2d(c, m, n);
+            return c.off;
+        case GPTQ_OP_REDUCED:
+            if (m < 1 || m > 65536 || n > LLL_MAX_N) return 0;
+            carve_reduced(c, m, n);
             return c.off;
         default:
             return 0;
@@ -625,6 +664,113 @@ GPTQ_API int gptq_2d_round(const float *X, int64_t m, int64_t n, const float *G,
                            int32_t *Z, float *err, void *workspace, size_t ws_bytes,
                            gptq_stream_t stream) {
     const int st = gptq_2d_round_body(X, m, n, G, H, Z, err, workspace, ws_bytes, stream);
+    return finish_call(st, stream);
+}
+
+static int gptq_quantize_layer_reduced_body(const void *W, int w_dtype, int64_t m, int64_t n,
+                                            const float *H, int bits, float lambda_rel,
+                                            uint32_t *codes, float *scales, uint8_t *zeros,
+                                            double *loss_out, int32_t *coef_out,
+                                            int64_t *stats_out, void *workspace, size_t ws_bytes,
+                                            gptq_stream_t stream) {
+    if (!W || !H || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
+    if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
+    if (m < 1 || m > 65536 || n < 1 || n > LLL_MAX_N) return GPTQ_ERR_ARG;
+    if (bits < 2 || bits > 8 || (n * bits) % 32) return GPTQ_ERR_ARG;
+    if (!(lambda_rel >= 0.f) || !isfinite(lambda_rel)) return GPTQ_ERR_ARG;
+    const size_t need = gptq_workspace_size(GPTQ_OP_REDUCED, m, n, 0, 0);
+    if (int st = check_ws(workspace, ws_bytes, need)) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    Carver c(workspace);
+    ReducedWs w = carve_reduced(c, m, n);
+    const int N = (int)n, M = (int)m;
+    const long long mn = m * n;
+    const int blocks = (int)std::min<long long>((std::max<long long>(mn, n * n) + 255) / 256, 148LL * 8);
+    if (cudaMemsetAsync(w.stats, 0, sizeof(long long) * REDUCED_STATS, s) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    // lambda, G' = (H + lambda I) / 2, its LLL reduction T (and T^-1) for GPTQ's column order
+    damp_mean_kernel<<<1, 1024, 0, s>>>(H, n, N, lambda_rel, w.lam);
+    GPTQ_CHECK_LAUNCH();
+    lll_prep_kernel<<<blocks, 256, 0, s>>>(H, n, N, w.lam, w.A, w.Gd);
+    GPTQ_CHECK_LAUNCH();
+    lll_kernel<<<1, LLL_THREADS, 0, s>>>(w.A, N, w.Bn, w.T, w.Ti, w.stats, 64LL * n * n + 4096,
+                                         0.75);
+    GPTQ_CHECK_LAUNCH();
+    lll_export_kernel<<<blocks, 256, 0, s>>>(w.T, w.Ti, N, w.Tf, w.Tif, w.stats);
+    GPTQ_CHECK_LAUNCH();
+    // G_red = T^T G' T
+    if (int st = gemm_f32(gemm_args<float, float>(N, N, N, w.Gd, n, 0, w.Tf, n, 0, w.A2, n, 1.f,
+                                                  0.f), s)) return st;
+    if (int st = gemm_f32(gemm_args<float, float>(N, N, N, w.Tf, n, 1, w.A2, n, 0, w.Gred, n, 1.f,
+                                                  0.f), s)) return st;
+    // per-channel grid and the grid coordinates in the reduced basis, u' = T^-1 u
+    if (w_dtype == GPTQ_BF16)
+        rowgrid_kernel<__nv_bfloat16><<<ceil_div(m, 8), 256, 0, s>>>(
+            static_cast<const __nv_bfloat16 *>(W), M, N, bits, scales, zeros, w.U);
+    else
+        rowgrid_kernel<float><<<ceil_div(m, 8), 256, 0, s>>>(static_cast<const float *>(W), M, N,
+                                                              bits, scales, zeros, w.U);
+    GPTQ_CHECK_LAUNCH();
+    if (int st = gemm_f32(gemm_args<float, float>(M, N, N, w.U, n, 0, w.Tif, n, 1, w.Up, n, 1.f,
+                                                  0.f), s)) return st;
+    // Babai in the reduced basis: one-sided adaptive rounding of u' under G_red (the two-sided
+    // wavefront with U_G = I)
+    TwoDWs &t = w.w2;
+    gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(t.UG, 0, t.Mp);
+    GPTQ_CHECK_LAUNCH();
+    if (int st = prepare_hinv_impl(w.Gred, N, 0.f, t.UH, t.Np, t.lam, t.fh, s, 0)) return st;
+    if (t.Np > n) {
+        gptq2d_pad_identity_kernel<<<64, 256, 0, s>>>(t.UH, n, t.Np);
+        GPTQ_CHECK_LAUNCH();
+    }
+    gptq2d_init_kernel<<<1184, 256, 0, s>>>(w.Up, M, N, t.Xw, t.Cacc, t.Mp, t.Np);
+    GPTQ_CHECK_LAUNCH();
+    Gptq2dArgs a;
+    a.Xw = t.Xw; a.Cacc = t.Cacc; a.E = t.E; a.F = t.F; a.UG = t.UG; a.UH = t.UH;
+    a.Z = w.Zi; a.err = nullptr; a.Mp = t.Mp; a.Np = t.Np; a.m = M; a.n = N;
+    a.MT = (int)(t.Mp / T2D); a.NT = (int)(t.Np / T2D);
+    if (int st = gptq2d_sweep(a, s)) return st;
+    if (coef_out &&
+        cudaMemcpyAsync(coef_out, w.Zi, sizeof(int32_t) * mn, cudaMemcpyDeviceToDevice, s) !=
+            cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    // back to the original coordinates: c = clip(T c'), codes, loss
+    int_to_float_kernel<<<blocks, 256, 0, s>>>(w.Zi, mn, w.U);
+    GPTQ_CHECK_LAUNCH();
+    if (int st = gemm_f32(gemm_args<float, float>(M, N, N, w.U, n, 0, w.Tf, n, 1, w.Cr, n, 1.f,
+                                                  0.f), s)) return st;
+    if (w_dtype == GPTQ_BF16)
+        reduced_codes_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(
+            w.Cr, static_cast<const __nv_bfloat16 *>(W), scales, zeros, M, N, bits, w.c8, w.D,
+            w.stats);
+    else
+        reduced_codes_kernel<float><<<blocks, 256, 0, s>>>(w.Cr, static_cast<const float *>(W),
+                                                           scales, zeros, M, N, bits, w.c8, w.D,
+                                                           w.stats);
+    GPTQ_CHECK_LAUNCH();
+    pack_codes_kernel<<<blocks, 256, 0, s>>>(w.c8, M, N, bits, codes);
+    GPTQ_CHECK_LAUNCH();
+    if (loss_out) {
+        // (w - w_hat)^T (H + lambda I) (w - w_hat) = 2 d G' d^T
+        if (int st = gemm_f32(gemm_args<float, float>(M, N, N, w.D, n, 0, w.Gd, n, 0, w.DH, n,
+                                                      2.f, 0.f), s)) return st;
+        refine_rowdot_kernel<<<ceil_div(m, 8), 256, 0, s>>>(w.D, w.DH, M, N, loss_out);
+        GPTQ_CHECK_LAUNCH();
+    }
+    if (stats_out &&
+        cudaMemcpyAsync(stats_out, w.stats, sizeof(long long) * REDUCED_STATS,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return GPTQ_ERR_CUDA;
+    return GPTQ_OK;
+}
+
+GPTQ_API int gptq_quantize_layer_reduced(const void *W, int w_dtype, int64_t m, int64_t n,
+                                         const float *H, int bits, float lambda_rel,
+                                         uint32_t *codes, float *scales, uint8_t *zeros,
+                                         double *loss_out, int32_t *coef_out, int64_t *stats_out,
+                                         void *workspace, size_t ws_bytes, gptq_stream_t stream) {
+    const int st = gptq_quantize_layer_reduced_body(W, w_dtype, m, n, H, bits, lambda_rel, codes,
+        scales, zeros, loss_out, coef_out, stats_out, workspace, ws_bytes, stream);
     return finish_call(st, stream);
 }
 

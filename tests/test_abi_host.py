@@ -22,7 +22,7 @@ def test_header_declares_the_boundary():
         "gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
         "gptq_quantize_layer_noalloc", "gptq_il_quantize_layer", "gptq_il_refine",
         "gptq_quantize_lowrank", "gptq_2d_round", "gptq_set_flags", "gptq_get_flags",
-        "gptq_kernel_times"])
+        "gptq_kernel_times", "gptq_quantize_layer_reduced"])
 
 
 def test_library_exports_every_declared_symbol():
@@ -223,3 +223,32 @@ def test_kernel_times_record_is_empty_and_checks_its_arguments():
     assert g.gptq_kernel_times(None, 3) == g.GPTQ_ERR_ARG
     assert g.gptq_kernel_times(arr, -1) == g.GPTQ_ERR_ARG
     assert g.kernel_times() == {}
+
+
+P1 = ctypes.c_void_p(256)
+
+
+@pytest.mark.parametrize("m,n,bits,lam,wdt", [
+    (0, 256, 4, 0.01, 1), (8, 0, 4, 0.01, 1), (8, 2049, 4, 0.01, 1), (8, 256, 1, 0.01, 1),
+    (8, 256, 9, 0.01, 1), (8, 100, 4, 0.01, 1), (8, 256, 4, -1.0, 1), (8, 256, 4, 0.01, 7)])
+def test_reduced_rejects_bad_arguments(m, n, bits, lam, wdt):
+    import post_weight_quantization_06_b200 as g
+    before = g.gptq_launch_count()
+    st = _lib().gptq_quantize_layer_reduced(P1, wdt, m, n, P1, bits, ctypes.c_float(lam), P1, P1,
+                                            P1, NULL, NULL, NULL, ctypes.c_void_p(1 << 20),
+                                            1 << 40, NULL)
+    assert st == -1
+    assert g.gptq_launch_count() == before
+
+
+def test_reduced_checks_its_workspace():
+    import post_weight_quantization_06_b200 as g
+    m, n = 64, 256
+    need = g.gptq_workspace_size(g.GPTQ_OP_REDUCED, m, n, 0, 0)
+    assert need > 0 and g.gptq_workspace_size(g.GPTQ_OP_REDUCED, m, 4096, 0, 0) == 0
+    before = g.gptq_launch_count()
+    st = _lib().gptq_quantize_layer_reduced(P1, 1, m, n, P1, 4, ctypes.c_float(0.01), P1, P1, P1,
+                                            NULL, NULL, NULL, ctypes.c_void_p(1 << 20), need - 1,
+                                            NULL)
+    assert st == -6
+    assert g.gptq_launch_count() == before

@@ -47,12 +47,13 @@ def test_noalloc_matches_workspace_entry_twice(wl, scale):
         held, free = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         g.gptq_quantize_layer_noalloc(L.W, U, L.bits, L.group_size, L.block_size, *out)
         g.gptq_sync_status()
-        for a, b in zip(ref, out):
-            assert torch.equal(a, b)
+        held_after, free_after = torch.cuda.memory_allocated(), torch.cuda.mem_get_info()[0]
         if call == 1:
             # the warm call takes no device memory: neither through torch nor from the driver
-            assert torch.cuda.memory_allocated() == held
-            assert torch.cuda.mem_get_info()[0] == free
+            assert held_after == held
+            assert free_after == free
+        for a, b in zip(ref, out):
+            assert torch.equal(a, b)
 
 
 def test_noalloc_rejects_layers_beyond_the_scratch():

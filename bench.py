@@ -249,21 +249,19 @@ def sweep_roofline(layer, sweep_ms: float, gemm) -> dict:
 
 
 def hessian_traffic(layer):
-    """DRAM bytes per Hessian launch from the committed ncu summary, for the full 2048x6144 /
-    262144-token workload only, and only while the kernel source is the one profiled."""
+    """DRAM bytes per Hessian launch from the committed one-pass ncu capture
+    (profiles/hessian_tc_traffic.json), for the full 2048x6144 / 262144-token workload only, and
+    only while the kernel source is the one profiled."""
     import hashlib
-    import re
     if (layer.n, layer.k) != (6144, 262144):
         return None
     try:
-        txt = open(os.path.join(ROOT, "profiles", "hessian_tc.md")).read()
-        traffic = int(re.search(r"traffic_bytes_per_launch:\s*(\d+)", txt).group(1))
-        src = re.search(r"kernel_source:\s*(\S+)", txt).group(1)
-        digest = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", txt).group(1)
-        current = hashlib.sha256(open(os.path.join(ROOT, src), "rb").read()).hexdigest()[:16]
-    except (OSError, AttributeError, ValueError):
+        rec = json.load(open(os.path.join(ROOT, "profiles", "hessian_tc_traffic.json")))
+        src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
+        current = hashlib.sha256(src).hexdigest()[:16]
+    except (OSError, KeyError, ValueError):
         return None
-    return traffic if current == digest else None
+    return int(rec["traffic_bytes_per_launch"]) if current == rec["kernel_source_sha256_16"] else None
 
 
 def run_e2e(g, layer, lp, steps, warmup, chunk_tokens=32768):

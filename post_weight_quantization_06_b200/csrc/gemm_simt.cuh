@@ -30,6 +30,7 @@ struct GemmArgs {
     int pdl;            // SIMT path: launch as a programmatic dependent of the stream's previous
                         // kernel (the launch overlaps that kernel's tail)
     const int *skip;    // when set and *skip != 0 the launch does nothing
+    const float *a_lo;  // A given as tf32 hi (A) and lo (a_lo, same layout): op(A) = A + a_lo
 };
 
 namespace simt {
@@ -191,6 +192,7 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.max_ctas = 0;
     p.pdl = 0;
     p.skip = nullptr;
+    p.a_lo = nullptr;
     return p;
 }
 

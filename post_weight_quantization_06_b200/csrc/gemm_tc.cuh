@@ -140,6 +140,7 @@ struct TcGemmParams {
     int c_tma;          // 1: beta is 0 or 1 and cmap covers C; slices may leave by tensor store /
                         // tensor add-reduction instead of a read-modify-write
     const int *skip;    // when set and *skip != 0 the launch does nothing
+    int a_split;        // 1: A comes split (amap: tf32 hi, alomap: lo); only B is converted
 };
 
 // Bulk tensor writes of one 32 x 32 slice from shared memory (128-byte swizzle) through the C
@@ -210,7 +211,8 @@ __device__ __forceinline__ void epi_load_c(const TcGemmParams &p, int row_base, 
 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-               const __grid_constant__ CUtensorMap cmap, TcGemmParams p) {
+               const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap alomap,
+               TcGemmParams p) {
     if (p.skip && *p.skip) return;   // before any barrier, TMEM or copy: every thread leaves
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
@@ -233,6 +235,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&amap)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&bmap)) : "memory");
         if (p.c_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&cmap)) : "memory");
+        if (p.a_split) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&alomap)) : "memory");
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&conv[s], CONV_WARPS);
@@ -269,12 +272,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         break;
                     }
                     unsigned char *st = base + slot * STAGE_BYTES;
-                    mbar_expect_tx(&full[slot], 2 * SLICE_BYTES);
+                    mbar_expect_tx(&full[slot], (p.a_split ? 3 : 2) * SLICE_BYTES);
                     if (p.a_mn) {
                         for (int q = 0; q < 4; ++q)
                             tma_load_2d(&amap, &full[slot], st + q * (BK * 128), ti * TILE + 32 * q, k0);
+                        if (p.a_split)
+                            for (int q = 0; q < 4; ++q)
+                                tma_load_2d(&alomap, &full[slot], st + SLICE_BYTES + q * (BK * 128),
+                                            ti * TILE + 32 * q, k0);
                     } else {
                         tma_load_2d(&amap, &full[slot], st, k0, ti * TILE);
+                        if (p.a_split) tma_load_2d(&alomap, &full[slot], st + SLICE_BYTES, k0, ti * TILE);
                     }
                     unsigned char *sb = st + 2 * SLICE_BYTES;
                     if (p.b_mn) {
@@ -356,17 +364,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     break;
                 }
                 unsigned char *st = base + slot * STAGE_BYTES;
-                // every thread splits CONV_PER float4 of each operand; all of its shared-memory
-                // loads go out first so that their latencies overlap
+                // every thread splits CONV_PER float4 of each operand (of B alone when A came
+                // split); all of its shared-memory loads go out first so that their latencies
+                // overlap
+                const int op0 = p.a_split ? 1 : 0;
                 float4 x[2][CONV_PER];
 #pragma unroll
                 for (int op = 0; op < 2; ++op) {
+                    if (op < op0) continue;
                     const float4 *hi = reinterpret_cast<const float4 *>(st + op * 2 * SLICE_BYTES);
 #pragma unroll
                     for (int u = 0; u < CONV_PER; ++u) x[op][u] = hi[cw * 32 + lane + u * CONV_WARPS * 32];
                 }
 #pragma unroll
                 for (int op = 0; op < 2; ++op) {
+                    if (op < op0) continue;
                     float4 *hi = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES);
                     float4 *lo = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES + SLICE_BYTES);
 #pragma unroll
@@ -541,9 +553,20 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
     static const bool force_simt = std::getenv("GPTQ_FORCE_SIMT_GEMM") != nullptr;
     const bool small = (long long)g.M * g.N < 128LL * 256 || g.K < 64;
+    // a split A on the SIMT path: C = alpha (A_hi + A_lo) B + beta C as two products
+    auto simt = [&]() -> int {
+        if (!g.a_lo) return gemm_simt(g, s);
+        GemmArgs<float, float> h = g;
+        h.a_lo = nullptr;
+        if (int st = gemm_simt(h, s)) return st;
+        h.A = g.a_lo;
+        h.beta = 1.f;
+        return gemm_simt(h, s);
+    };
     if (small || !tcg::tc_eligible(g.A, g.lda, g.B, g.ldb) ||
+        (g.a_lo && !tcg::tc_eligible(g.a_lo, g.lda, g.B, g.ldb)) ||
         (reinterpret_cast<uintptr_t>(g.C) & 3u) || force_simt)
-        return gemm_simt(g, s);
+        return simt();
     tcg::TcGemmParams p;
     p.M = g.M; p.N = g.N; p.K = g.K;
     p.C = g.C; p.ldc = g.ldc;
@@ -561,7 +584,13 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
                              : tcg::make_map_f32(&am, g.A, g.M, g.K, g.lda, 32, tcg::TILE, false);
     const bool ok_b = p.b_mn ? tcg::make_map_f32(&bm, g.B, g.K, g.N, g.ldb, 32, 32, true)
                              : tcg::make_map_f32(&bm, g.B, g.N, g.K, g.ldb, 32, tcg::TILE, false);
-    if (!ok_a || !ok_b) return gemm_simt(g, s);
+    CUtensorMap alm;
+    p.a_split = g.a_lo ? 1 : 0;
+    const bool ok_al = !g.a_lo ||
+        (p.a_mn ? tcg::make_map_f32(&alm, g.a_lo, g.K, g.M, g.lda, 32, 32, true)
+                : tcg::make_map_f32(&alm, g.a_lo, g.M, g.K, g.lda, 32, tcg::TILE, false));
+    if (!ok_a || !ok_b || !ok_al) return simt();
+    if (!g.a_lo) alm = am;   // not read
     // C through a tensor map when beta is 0 or 1 and C's base and pitch allow it
     static const bool rmw_only = std::getenv("GPTQ_GEMM_RMW_EPILOGUE") != nullptr;
     p.c_tma = !rmw_only && (g.beta == 0.f || g.beta == 1.f) &&
@@ -574,7 +603,7 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
     GPTQ_SMEM_LIMIT(tcg::gemm_tc_kernel, tcg::SMEM_BYTES);
     KtSpan span(s, g.skip != nullptr);
-    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, cm, p);
+    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, cm, alm, p);
     const int st = launch_status();
     span.done(KT_TC, g);
     return st;

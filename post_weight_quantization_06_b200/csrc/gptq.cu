@@ -43,7 +43,7 @@ inline FactorWs carve_factor(Carver &c, long long n) {
 }
 
 struct QuantWs {
-    float *Wc, *Err;
+    float *Wc, *Err, *Err_lo;
 };
 // Err holds the errors of one outer block of the two-level lazy update: m x OB with
 // OB <= min(QUANT_OUTER_MAX, n).
@@ -52,6 +52,7 @@ inline QuantWs carve_quant(Carver &c, long long m, long long N, int B) {
     w.Wc = c.take<float>((size_t)m * N);
     const long long ob = N < QUANT_OUTER_MAX ? N : QUANT_OUTER_MAX;
     w.Err = c.take<float>((size_t)m * (ob > B ? ob : B));
+    w.Err_lo = c.take<float>((size_t)m * (ob > B ? ob : B));
     return w;
 }
 
@@ -450,7 +451,7 @@ static int gptq_quantize_layer_body(const void *W, int w_dtype, int64_t m, int64
     QuantWs w = carve_quant(c, m, n, block_size);
     if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
     return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
-                       codes, scales, zeros, loss_out, w.Err, s);
+                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, s);
 }
 
 GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
@@ -481,7 +482,7 @@ static int gptq_quantize_layer_noalloc_body(const void *W, int w_dtype, int64_t 
     QuantWs w = carve_quant(c, m, n, block_size);
     if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
     return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
-                       codes, scales, zeros, loss_out, w.Err, s);
+                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, s);
 }
 
 GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
@@ -522,7 +523,7 @@ static int gptq_il_quantize_layer_body(const void *W, int w_dtype, int64_t m, in
     }
     if (int st = init_work(W, w_dtype, m, (int)n, w.q.Wc, N, (int)N, s)) return st;
     if (int st = sweep_layer(w.q.Wc, N, (int)m, (int)n, (int)N, w.Uaug, N, bits, group_size,
-                             block_size, codes, scales, zeros, loss_out, w.q.Err, s))
+                             block_size, codes, scales, zeros, loss_out, w.q.Err, w.q.Err_lo, s))
         return st;
     if (r > 0) {
         extract_R_kernel<<<592, 256, 0, s>>>(w.q.Wc, N, (int)m, (int)n, r, R);

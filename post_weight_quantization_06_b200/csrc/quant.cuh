@@ -44,8 +44,9 @@ struct ColloopArgs {
     float *scales;      // m x G
     uint8_t *zeros;     // m x G
     int G;
-    float *err;         // errors of this panel: m x B block at err (row stride lde)
-    long long lde;
+    float *err;         // errors of this panel: m x B block at err (row stride lde), as the
+    float *err_lo;      // tf32 pair hi = tf32(e) (err), lo = tf32(e - hi) (err_lo) that the
+    long long lde;      // lazy update's tensor-core product takes without converting them
     double *loss;       // m or nullptr
 };
 
@@ -105,8 +106,7 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
     const int maxq = (1 << a.bits) - 1;
     const float fmaxq = (float)maxq;
     const int row0 = (blockIdx.x * nwarps + warp) * ROWS;
-    float w[ROWS][NSLOT], ev[ROWS][NSLOT];
-    float cv[ROWS][NSLOT];   // codes kept as floats until the panel is done
+    float w[ROWS][NSLOT];
     float s[ROWS], is[ROWS], z[ROWS];
     bool rv[ROWS];
 #pragma unroll
@@ -117,8 +117,6 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
 #pragma unroll
         for (int q = 0; q < NSLOT; ++q) {
             w[r][q] = rv[r] ? a.Wc[(long long)row * a.ldw + j0 + 32 * q + lane] : 0.f;
-            ev[r][q] = 0.f;
-            cv[r][q] = 0.f;
         }
     }
     if (async_u) asm volatile("cp.async.wait_group 0;\n" ::: "memory");
@@ -163,8 +161,18 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
         }
     }
 
+    // The panel's slots one after the other, the current one always in register slot 0: after
+    // each slot the registers rotate down by one, so the loop over slots is a real loop whose
+    // body (32 column steps, partly unrolled) is fetched once and reused NSLOT times.
+    uint8_t *cb = cbuf + warp * ROWS * B;
+    double lacc[ROWS];
 #pragma unroll
+    for (int r = 0; r < ROWS; ++r) lacc[r] = 0.0;
+#pragma unroll 1
     for (int q = 0; q < NSLOT; ++q) {
+        float cvc[ROWS], evc[ROWS];
+#pragma unroll
+        for (int r = 0; r < ROWS; ++r) { cvc[r] = 0.f; evc[r] = 0.f; }
 #pragma unroll 4
         for (int o = 0; o < 32; ++o) {
             const int t = 32 * q + o;
@@ -174,11 +182,11 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
                 for (int r = 0; r < ROWS; ++r) {
                     float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-                    for (int q2 = 0; q2 < NSLOT; ++q2) {
-                        const int col = 32 * q2 + lane;
-                        if (q2 >= q && col >= t && col < t + gs) {
-                            mn = fminf(mn, w[r][q2]);
-                            mx = fmaxf(mx, w[r][q2]);
+                    for (int sl = 0; sl < NSLOT; ++sl) {
+                        const int col = 32 * (q + sl) + lane;
+                        if (q + sl < NSLOT && col >= t && col < t + gs) {
+                            mn = fminf(mn, w[r][sl]);
+                            mx = fmaxf(mx, w[r][sl]);
                         }
                     }
                     mn = warp_min(mn);
@@ -192,42 +200,45 @@ __global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
                 }
             }
             const float ut = invd[t];
+            const float *urow = Us + t * B + 32 * q + lane;
 #pragma unroll
             for (int r = 0; r < ROWS; ++r) {
-                const float wt = __shfl_sync(0xffffffffu, w[r][q], o);
+                const float wt = __shfl_sync(0xffffffffu, w[r][0], o);
                 const float v = fmaf(wt, is[r], z[r]);
                 const float c = fminf(fmaxf(rintf(v), 0.f), fmaxq);
                 const float wq = s[r] * (c - z[r]);
                 const float e = (wt - wq) * ut;
                 if (lane == o) {
-                    cv[r][q] = c;
-                    ev[r][q] = e;
+                    cvc[r] = c;
+                    evc[r] = e;
                 }
+                if (lane > o) w[r][0] = fmaf(-e, urow[0], w[r][0]);
 #pragma unroll
-                for (int q2 = q; q2 < NSLOT; ++q2) {
-                    const int col = 32 * q2 + lane;
-                    if (q2 > q || lane > o) w[r][q2] = fmaf(-e, Us[t * B + col], w[r][q2]);
-                }
+                for (int sl = 1; sl < NSLOT; ++sl)
+                    if (q + sl < NSLOT) w[r][sl] = fmaf(-e, urow[32 * sl], w[r][sl]);
             }
         }
-    }
-
-    // errors of the panel (for the lazy update), loss, packed codes
-    uint8_t *cb = cbuf + warp * ROWS * B;
+        // slot q is final: its errors (for the lazy update), codes and loss share
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        const int row = row0 + r;
+        for (int r = 0; r < ROWS; ++r) {
+            const int row = row0 + r;
+            if (rv[r]) {
+                const float eh = tcg::to_tf32(evc[r]);
+                a.err[(long long)row * a.lde + 32 * q + lane] = eh;
+                a.err_lo[(long long)row * a.lde + 32 * q + lane] = tcg::to_tf32(evc[r] - eh);
+            }
+            cb[r * B + 32 * q + lane] = (uint8_t)(int)cvc[r];
+            lacc[r] += (double)evc[r] * (double)evc[r];
 #pragma unroll
-        for (int q = 0; q < NSLOT; ++q) {
-            if (rv[r]) a.err[(long long)row * a.lde + 32 * q + lane] = ev[r][q];
-            cb[r * B + 32 * q + lane] = (uint8_t)(int)cv[r][q];
+            for (int sl = 0; sl + 1 < NSLOT; ++sl) w[r][sl] = w[r][sl + 1];
+            w[r][NSLOT - 1] = 0.f;
         }
-        if (a.loss) {
-            // the panel's share of the loss: each lane's own columns, then the warp's sum
-            double l = 0.0;
+    }
+    if (a.loss) {
 #pragma unroll
-            for (int q = 0; q < NSLOT; ++q) l += (double)ev[r][q] * (double)ev[r][q];
-            l = warp_sum_d(l);
+        for (int r = 0; r < ROWS; ++r) {
+            const int row = row0 + r;
+            const double l = warp_sum_d(lacc[r]);
             if (lane == 0 && rv[r]) {
                 if (j0 == 0) a.loss[row] = l;
                 else a.loss[row] += l;
@@ -303,7 +314,7 @@ inline int outer_block(int n, int gs, int B) {
 // products with K = B. Err holds m x OB floats.
 inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const float *U,
                        long long ldu, int bits, int group_size, int B, uint32_t *codes,
-                       float *scales, uint8_t *zeros, double *loss, float *Err,
+                       float *scales, uint8_t *zeros, double *loss, float *Err, float *Err_lo,
                        cudaStream_t s) {
     KtStageScope stage(GPTQ_KT_SWEEP);
     const int gs = group_size ? group_size : n;
@@ -319,6 +330,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
         for (int j0 = o0; j0 < o1; j0 += B) {
             a.j0 = j0;
             a.err = Err + (j0 - o0);
+            a.err_lo = Err_lo + (j0 - o0);
             int st;
             switch (B) {
                 case 32: st = colloop_launch<1>(a, s); break;
@@ -332,6 +344,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
                 auto p = gemm_args<float, float>(m, o1 - j1, B, Err + (j0 - o0), OB, 0,
                                                  U + (long long)j0 * ldu + j1, ldu, 0, Wc + j1,
                                                  ldw, -1.f, 1.f);
+                p.a_lo = Err_lo + (j0 - o0);
                 if (int st2 = gemm_f32(p, s)) return st2;
             }
         }
@@ -340,6 +353,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
             auto p = gemm_args<float, float>(m, N - o1, o1 - o0, Err, OB, 0,
                                              U + (long long)o0 * ldu + o1, ldu, 0, Wc + o1, ldw,
                                              -1.f, 1.f);
+            p.a_lo = Err_lo;
             if (int st2 = gemm_f32(p, s)) return st2;
         }
     }

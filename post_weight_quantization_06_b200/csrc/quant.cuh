@@ -31,7 +31,8 @@ __global__ void init_work_kernel(const TW *W, long long m, int n, float *Wc, lon
 }
 
 struct ColloopArgs {
-    float *Wc;          // m x N working weights (row stride ldw)
+    float *Wc;          // m x N working weights (row stride ldw); a finished panel keeps
+                        // its codes there as bytes (first CPL bytes of each CPL-column slot)
     long long ldw;
     const float *U;     // n x N upper factor rows (row stride ldu)
     long long ldu;
@@ -39,8 +40,6 @@ struct ColloopArgs {
     int j0;             // first column of this panel
     int bits;
     int gs;             // group length (n when there is one group per row)
-    uint32_t *codes;    // m x (n*bits/32)
-    long long ldcodes;
     float *scales;      // m x G
     uint8_t *zeros;     // m x G
     int G;
@@ -61,225 +60,366 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float fmaxq,
     z = fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.f), fmaxq);
 }
 
-// One CTA = 8 warps; one warp = ROWS rows; lane l owns columns l, l+32, ... of the panel.
-// The panel's U block (B x B) and 1/U_jj sit in shared memory. Per column t: the owner
-// lane's value is broadcast by shuffle, every lane evaluates the rounding of that column
-// for its rows (the same value on all lanes), and each lane applies -e * U[t, col] to the
-// columns it owns that come after t.
-template <int NSLOT, int ROWS>
-__global__ __launch_bounds__(256) void colloop_kernel(ColloopArgs a) {
-    constexpr int B = 32 * NSLOT;
+constexpr int COLLOOP_THREADS = 128;
+
+// One warp = 32 / LPR rows; the LPR = B / CPL lanes of a row each hold CPL (16) consecutive
+// columns of the panel in registers (lane k of the row: columns CPL k .. CPL k + CPL-1, "slot"
+// k), so that the rounding of a column is evaluated by LPR lanes per row and every lane applies
+// at most CPL updates per column. The panel's U block sits in shared memory (rows from their
+// diagonal slot on, zeros to the left of it; 4 floats of padding after every slot, so that the
+// lanes of a row, which read 16 bytes each from their own slot, hit different banks). Per
+// column t = CPL q + o: the owner lane (k = q) broadcasts register o to its row's lanes by
+// shuffle, every lane of the row evaluates the rounding, and each lane applies -e * U[t, col]
+// to its own columns after t, the next column first (its new value is the next step's
+// shuffle). Lanes without work in a step multiply by a zero error instead of branching (U is
+// finite, the zeros left of the diagonal included), so the warp never diverges. The owner keeps
+// e in the column's register, so that at the end of the panel every register holds the error
+// of its column; the codes go to the panel's own columns of Wc as bytes (those columns are
+// final) and are bit-packed once after the sweep. SMALLG: groups shorter than a slot, whose
+// boundaries fall inside it.
+constexpr int COLLOOP_CPL = 16;  // columns per lane
+template <int B>
+struct ColloopShape {
+    static constexpr int CPL = COLLOOP_CPL;
+    static constexpr int LPR = B / CPL;        // lanes per row
+    static constexpr int RPW = 32 / LPR;       // rows per warp
+    static constexpr int LDU = B + 4 * LPR;    // padded row of the U block, in floats
+    static __host__ __device__ constexpr int col(int c) { return c + 4 * (c / CPL); }
+};
+
+template <int B, bool SMALLG>
+__global__ __launch_bounds__(COLLOOP_THREADS, 1) void colloop_kernel(ColloopArgs a) {
+    using S = ColloopShape<B>;
+    constexpr int CPL = S::CPL, LPR = S::LPR, RPW = S::RPW, LDU = S::LDU;
     extern __shared__ float sm[];
     float *Us = sm;
-    float *invd = Us + B * B;
-    uint8_t *cbuf = reinterpret_cast<uint8_t *>(invd + B);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nwarps = blockDim.x >> 5;
+    const int k = lane % LPR;
+    const int row = (blockIdx.x * nwarps + warp) * RPW + lane / LPR;
+    const bool rv = row < a.m;
     const int j0 = a.j0;
-    // U block load: with 16-byte aligned rows all of it goes out at once as cp.async (the
-    // weight rows below load meanwhile); otherwise eight plain loads in flight per thread
+    // U block: slot q's rows (CPL q .. CPL q + CPL-1) hold zeros left of column CPL q; from there on
+    // cp.async when the rows are 16-byte aligned, else plain loads
+    for (int q = 1; q < LPR; ++q) {
+        const int f4 = CPL * q / 4;  // float4s of a row left of its diagonal slot
+        for (int c = tid; c < CPL * f4; c += blockDim.x) {
+            const int rr = CPL * q + c / f4, cc = (c % f4) * 4;
+            *reinterpret_cast<float4 *>(Us + rr * LDU + S::col(cc)) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    }
     const bool async_u = ((reinterpret_cast<uintptr_t>(a.U) | (uintptr_t)(a.ldu * 4)) & 15u) == 0;
     if (async_u) {
-        for (int c = tid; c < B * B / 4; c += blockDim.x) {
-            const int row = c / (B / 4), q4 = (c % (B / 4)) * 4;
-            const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(Us + row * B + q4));
-            const float *src = a.U + (long long)(j0 + row) * a.ldu + j0 + q4;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+#pragma unroll
+        for (int q = 0; q < LPR; ++q) {
+            const int w4 = (B - CPL * q) / 4;  // float4s per row from the diagonal slot on
+            for (int c = tid; c < CPL * w4; c += blockDim.x) {
+                const int rr = CPL * q + c / w4, cc = CPL * q + (c % w4) * 4;
+                const unsigned d =
+                    static_cast<unsigned>(__cvta_generic_to_shared(Us + rr * LDU + S::col(cc)));
+                const float *src = a.U + (long long)(j0 + rr) * a.ldu + j0 + cc;
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
+            }
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
     } else {
-        for (int base = tid; base < B * B; base += 8 * blockDim.x) {
-            float v[8];
+        for (int idx = tid; idx < B * B; idx += blockDim.x) {
+            const int rr = idx / B, cc = idx % B;
+            if (cc >= (rr & ~(CPL - 1)))
+                Us[rr * LDU + S::col(cc)] = a.U[(long long)(j0 + rr) * a.ldu + j0 + cc];
+        }
+    }
+    // the next panel's U block into L2 while this panel runs (one CTA asks for it)
+    if (blockIdx.x == 0 && j0 + 2 * B <= a.n) {
+        for (int rr = tid; rr < B; rr += blockDim.x) {
+            const float *p = a.U + (long long)(j0 + B + rr) * a.ldu + j0 + B;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int idx = base + u * blockDim.x;
-                v[u] = idx < B * B ? a.U[(long long)(j0 + idx / B) * a.ldu + j0 + idx % B] : 0.f;
-            }
+            for (int c = 0; c < B; c += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + c));
+        }
+    }
+
+    float w[CPL];
+    {
+        const float *src = a.Wc + (long long)row * a.ldw + j0 + CPL * k;
+        const bool vec = ((reinterpret_cast<uintptr_t>(a.Wc) | (uintptr_t)(a.ldw * 4)) & 15u) == 0;
+        if (rv && vec) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int idx = base + u * blockDim.x;
-                if (idx < B * B) Us[idx] = v[u];
+            for (int j = 0; j < CPL / 4; ++j) {
+                const float4 v = reinterpret_cast<const float4 *>(src)[j];
+                w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
             }
+        } else {
+#pragma unroll
+            for (int r = 0; r < CPL; ++r) w[r] = rv ? src[r] : 0.f;
         }
     }
 
     const int maxq = (1 << a.bits) - 1;
     const float fmaxq = (float)maxq;
-    const int row0 = (blockIdx.x * nwarps + warp) * ROWS;
-    float w[ROWS][NSLOT];
-    float s[ROWS], is[ROWS], z[ROWS];
-    bool rv[ROWS];
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        const int row = row0 + r;
-        rv[r] = row < a.m;
-        s[r] = 1.f; is[r] = 1.f; z[r] = 0.f;
-#pragma unroll
-        for (int q = 0; q < NSLOT; ++q) {
-            w[r][q] = rv[r] ? a.Wc[(long long)row * a.ldw + j0 + 32 * q + lane] : 0.f;
+    const int gs = a.gs;
+    const bool groups_in_panel = gs <= B;  // then B % gs == 0
+    const int gmask = groups_in_panel ? gs - 1 : 0;
+    float s = 1.f, is = 1.f, z = 0.f;
+    if (!groups_in_panel) {
+        // one group spans several panels; its grid was computed at its first panel
+        const int g = j0 / gs;
+        if (rv) {
+            s = a.scales[(long long)row * a.G + g];
+            z = (float)a.zeros[(long long)row * a.G + g];
+            is = __frcp_rn(s);
         }
     }
+
+    // grid of the group that starts at panel column t, from the current weights of its columns
+    auto group_grid = [&](int t) {
+        float mn = INFINITY, mx = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < CPL; ++r) {
+            if ((unsigned)(CPL * k + r - t) < (unsigned)gs) {
+                mn = fminf(mn, w[r]);
+                mx = fmaxf(mx, w[r]);
+            }
+        }
+#pragma unroll
+        for (int x = 1; x < LPR; x <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, x));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, x));
+        }
+        grid_from_range(mn, mx, fmaxq, s, is, z);
+        if (k == 0 && rv) {
+            const int g = (j0 + t) / gs;
+            a.scales[(long long)row * a.G + g] = s;
+            a.zeros[(long long)row * a.G + g] = (uint8_t)z;
+        }
+    };
+
+    // 1 / U[t, t] for every row of the block, once it has arrived
     if (async_u) asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
-    for (int t = tid; t < B; t += blockDim.x) invd[t] = 1.0f / Us[t * B + t];
+    float *invd = Us + B * LDU;
+    for (int t = tid; t < B; t += blockDim.x) invd[t] = __frcp_rn(Us[t * LDU + S::col(t)]);
     __syncthreads();
-    const int gs = a.gs;
-    const bool groups_in_panel = gs <= B;  // then B % gs == 0, so gs is a power of two
-    const int gmask = groups_in_panel ? gs - 1 : 0;
-    if (!groups_in_panel) {
-        const int g = j0 / gs;
-        if (j0 % gs == 0) {
-            const int cend = min(j0 + gs, a.n);
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                const int row = row0 + r;
-                float mn = INFINITY, mx = -INFINITY;
-                if (rv[r])
-                    for (int c = j0 + lane; c < cend; c += 32) {
-                        const float x = a.Wc[(long long)row * a.ldw + c];
-                        mn = fminf(mn, x);
-                        mx = fmaxf(mx, x);
-                    }
-                mn = warp_min(mn);
-                mx = warp_max(mx);
-                grid_from_range(mn, mx, fmaxq, s[r], is[r], z[r]);
-                if (lane == 0 && rv[r]) {
-                    a.scales[(long long)row * a.G + g] = s[r];
-                    a.zeros[(long long)row * a.G + g] = (uint8_t)z[r];
-                }
-            }
-        } else {
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                const int row = row0 + r;
-                if (rv[r]) {
-                    s[r] = a.scales[(long long)row * a.G + g];
-                    z[r] = (float)a.zeros[(long long)row * a.G + g];
-                    is[r] = __frcp_rn(s[r]);
-                }
-            }
-        }
-    }
 
-    // The panel's slots one after the other, the current one always in register slot 0: after
-    // each slot the registers rotate down by one, so the loop over slots is a real loop whose
-    // body (32 column steps, partly unrolled) is fetched once and reused NSLOT times.
-    uint8_t *cb = cbuf + warp * ROWS * B;
-    double lacc[ROWS];
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) lacc[r] = 0.0;
+    // Rounding with the magic constant 1.5 * 2^23: fmaf(w, 1/s, z + MAGIC) - (z + MAGIC) is the
+    // product w/s + z rounded once, to the nearest integer with ties to even (|w/s + z| < 2^22;
+    // anything larger clamps the same way), minus z; clamped to [-z, maxq - z] it is c - z.
+    constexpr float MAGIC = 12582912.f;
+    // With DEFER the updates of column t's error to the lane's other columns are applied in the
+    // next step, behind that step's chain (its rounding, the next column's update and shuffle):
+    // only the column the next shuffle reads needs them first. Groups shorter than a slot
+    // (SMALLG) read the registers between steps and take every update at once instead.
+    constexpr bool DEFER = !SMALLG;
+    uint32_t cw[CPL / 4] = {};  // codes of this lane's columns, one byte each
+    const int src_base = lane & ~(LPR - 1);
+    float wt = __shfl_sync(0xffffffffu, w[0], src_base);
 #pragma unroll 1
-    for (int q = 0; q < NSLOT; ++q) {
-        float cvc[ROWS], evc[ROWS];
+    for (int q = 0; q < LPR; ++q) {
+        const int src = src_base | q;
+        const bool own = k == q, after = k >= q, upto = k > q;
+        const bool last = q + 1 == LPR;
+        const float *urow = Us + CPL * q * LDU + S::col(CPL * k);  // row CPL q, this lane's slot
+        if (groups_in_panel && ((CPL * q) & gmask) == 0) group_grid(CPL * q);
+        const float zm = z + MAGIC, nz = -z, hz = fmaxq - z;
+        float uts[CPL];  // 1 / U[t, t] for the slot's columns
 #pragma unroll
-        for (int r = 0; r < ROWS; ++r) { cvc[r] = 0.f; evc[r] = 0.f; }
-#pragma unroll 4
+        for (int j = 0; j < CPL / 4; ++j) {
+            const float4 x = reinterpret_cast<const float4 *>(invd + CPL * q)[j];
+            uts[4 * j] = x.x; uts[4 * j + 1] = x.y; uts[4 * j + 2] = x.z; uts[4 * j + 3] = x.w;
+        }
+        float4 un[CPL / 4];
+#pragma unroll
+        for (int j = 0; j < CPL / 4; ++j) un[j] = reinterpret_cast<const float4 *>(urow)[j];
+        float up[CPL];            // the previous step's row of U (DEFER)
+        float eap = 0.f, eup = 0.f;  // and its masked errors
+#pragma unroll
+        for (int o = 0; o < CPL; ++o) {
+            if (SMALLG && o > 0 && groups_in_panel && (o & gmask) == 0) group_grid(CPL * q + o);
+            const float zmo = SMALLG ? z + MAGIC : zm, nzo = SMALLG ? -z : nz,
+                        hzo = SMALLG ? fmaxq - z : hz;
+            const float ut = uts[o];
+            float u[CPL];
+#pragma unroll
+            for (int j = 0; j < CPL / 4; ++j) {
+                u[4 * j] = un[j].x; u[4 * j + 1] = un[j].y; u[4 * j + 2] = un[j].z; u[4 * j + 3] = un[j].w;
+            }
+            if (o + 1 < CPL) {
+                // the next row of U while this column is rounded
+#pragma unroll
+                for (int j = 0; j < CPL / 4; ++j)
+                    un[j] = reinterpret_cast<const float4 *>(urow + (o + 1) * LDU)[j];
+            }
+            const int rn = (o + 1) & (CPL - 1);  // the column the next shuffle reads
+            if (DEFER && o > 0) w[rn] = fmaf(-(rn > o - 1 ? eap : eup), up[rn], w[rn]);
+            // its multiplier, scaled by 1 / U[t, t] and masked to the lanes that hold it still
+            // unquantized (off the chain: it waits only for U)
+            const float un_next = ((o + 1 < CPL) ? after : upto) ? u[rn] * ut : 0.f;
+            const float d = fminf(fmaxf(fmaf(wt, is, zmo) - zmo, nzo), hzo);  // c - z
+            const float e1 = fmaf(-s, d, wt);                                 // w_t - q_t
+            // the next column first: its value is the next step's shuffle (it takes
+            // e1 * (U[t, col] / U[t, t]), the other columns (e1 / U[t, t]) * U[t, col]: the same
+            // product, rounded in another order)
+            w[rn] = fmaf(-e1, un_next, w[rn]);
+            if (o + 1 < CPL) wt = __shfl_sync(0xffffffffu, w[rn], src);
+            else if (!last) wt = __shfl_sync(0xffffffffu, w[0], src + 1);
+            if (DEFER && o > 0) {
+#pragma unroll
+                for (int r = 0; r < CPL; ++r) {
+                    if (r == rn || r == o) continue;  // o: the previous step's next column
+                    w[r] = fmaf(-(r > o - 1 ? eap : eup), up[r], w[r]);
+                }
+            }
+            const float e = e1 * ut;
+            const float ea = after ? e : 0.f;  // for this lane's columns after t
+            const float eu = upto ? e : 0.f;   // for its columns up to t
+            if (!DEFER) {
+#pragma unroll
+                for (int r = 0; r < CPL; ++r) {
+                    if (r == rn) continue;
+                    w[r] = fmaf(-(r > o ? ea : eu), u[r], w[r]);
+                }
+            }
+            w[o] = own ? e : w[o];
+            const uint32_t code = __float_as_uint(d + zmo) & 0xffu;  // MAGIC + c
+            cw[o >> 2] |= (own ? code : 0u) << (8 * (o & 3));
+            if (DEFER) {
+                eap = ea;
+                eup = eu;
+#pragma unroll
+                for (int r = 0; r < CPL; ++r) up[r] = u[r];
+            }
+        }
+        if (DEFER) {
+            // the slot's last column reaches the lane's other columns before the next slot
+#pragma unroll
+            for (int r = 1; r < CPL; ++r) w[r] = fmaf(-eup, up[r], w[r]);
+        }
+    }
+
+    // the registers now hold the panel's errors: tf32 pairs for the lazy update, their squares
+    // for the loss; the codes go to the first CPL bytes of this lane's CPL columns of Wc
+    float l4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < CPL; ++r) l4[r & 3] = fmaf(w[r], w[r], l4[r & 3]);
+    double l = ((double)l4[0] + (double)l4[1]) + ((double)l4[2] + (double)l4[3]);
+#pragma unroll
+    for (int x = 1; x < LPR; x <<= 1) l += __shfl_xor_sync(0xffffffffu, l, x);
+    if (!rv) return;
+    float *eh = a.err + (long long)row * a.lde + CPL * k;
+    float *el = a.err_lo + (long long)row * a.lde + CPL * k;
+    uint32_t *cdst = reinterpret_cast<uint32_t *>(a.Wc + (long long)row * a.ldw + j0 + CPL * k);
+    const bool vec = ((reinterpret_cast<uintptr_t>(a.err) | reinterpret_cast<uintptr_t>(a.err_lo) |
+                       (uintptr_t)(a.lde * 4) | reinterpret_cast<uintptr_t>(a.Wc) |
+                       (uintptr_t)(a.ldw * 4)) & 15u) == 0;
+    if (vec) {
+#pragma unroll
+        for (int j = 0; j < CPL / 4; ++j) {
+            float4 h, lo;
+            h.x = tcg::to_tf32(w[4 * j]);     lo.x = tcg::to_tf32(w[4 * j] - h.x);
+            h.y = tcg::to_tf32(w[4 * j + 1]); lo.y = tcg::to_tf32(w[4 * j + 1] - h.y);
+            h.z = tcg::to_tf32(w[4 * j + 2]); lo.z = tcg::to_tf32(w[4 * j + 2] - h.z);
+            h.w = tcg::to_tf32(w[4 * j + 3]); lo.w = tcg::to_tf32(w[4 * j + 3] - h.w);
+            reinterpret_cast<float4 *>(eh)[j] = h;
+            reinterpret_cast<float4 *>(el)[j] = lo;
+        }
+        if constexpr (CPL == 16) *reinterpret_cast<uint4 *>(cdst) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        else if constexpr (CPL == 8) *reinterpret_cast<uint2 *>(cdst) = make_uint2(cw[0], cw[1]);
+        else for (int j = 0; j < CPL / 4; ++j) cdst[j] = cw[j];
+    } else {
+#pragma unroll
+        for (int r = 0; r < CPL; ++r) {
+            const float h = tcg::to_tf32(w[r]);
+            eh[r] = h;
+            el[r] = tcg::to_tf32(w[r] - h);
+        }
+#pragma unroll
+        for (int j = 0; j < CPL / 4; ++j) cdst[j] = cw[j];
+    }
+    if (a.loss && k == 0) {
+        if (j0 == 0) a.loss[row] = l;
+        else a.loss[row] += l;
+    }
+}
+
+// Bit-packs the codes that the column loop left as bytes at the start of every cpl-column slot
+// of Wc (the codes of columns cpl*i .. cpl*i + cpl-1 in the first cpl bytes of Wc[row, cpl*i];
+// cpl = 4, 8, 16 or 32). One thread per row and 32 columns: their 32 codes fill exactly `bits`
+// words of the packed row (code c at bits [c * bits, (c + 1) * bits) of the row's stream,
+// little-endian words).
+__global__ void pack_sweep_codes_kernel(const float *Wc, long long ldw, long long m, int n,
+                                        int bits, int cpl, uint32_t *codes, long long ldcodes) {
+    const int chunks = n / 32;
+    const long long total = m * chunks;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const long long row = idx / chunks;
+        const int ch = (int)(idx % chunks);
+        const uint32_t *src = reinterpret_cast<const uint32_t *>(Wc + row * ldw + 32 * ch);
+        uint32_t cw[8];  // codes 4j .. 4j+3: word (4j mod cpl) / 4 of the slot at 4j - 4j mod cpl
+#pragma unroll
+        for (int j = 0; j < 8; ++j) cw[j] = src[((4 * j) & ~(cpl - 1)) + (((4 * j) & (cpl - 1)) >> 2)];
+        uint32_t *dst = codes + row * ldcodes + (long long)ch * bits;
+        unsigned long long buf = 0;
+        int nb = 0, wi = 0;
+#pragma unroll
         for (int o = 0; o < 32; ++o) {
-            const int t = 32 * q + o;
-            if (groups_in_panel && (t & gmask) == 0) {
-                const int g = (j0 + t) / gs;
-#pragma unroll
-                for (int r = 0; r < ROWS; ++r) {
-                    float mn = INFINITY, mx = -INFINITY;
-#pragma unroll
-                    for (int sl = 0; sl < NSLOT; ++sl) {
-                        const int col = 32 * (q + sl) + lane;
-                        if (q + sl < NSLOT && col >= t && col < t + gs) {
-                            mn = fminf(mn, w[r][sl]);
-                            mx = fmaxf(mx, w[r][sl]);
-                        }
-                    }
-                    mn = warp_min(mn);
-                    mx = warp_max(mx);
-                    grid_from_range(mn, mx, fmaxq, s[r], is[r], z[r]);
-                    if (lane == 0 && rv[r]) {
-                        const int row = row0 + r;
-                        a.scales[(long long)row * a.G + g] = s[r];
-                        a.zeros[(long long)row * a.G + g] = (uint8_t)z[r];
-                    }
-                }
-            }
-            const float ut = invd[t];
-            const float *urow = Us + t * B + 32 * q + lane;
-#pragma unroll
-            for (int r = 0; r < ROWS; ++r) {
-                const float wt = __shfl_sync(0xffffffffu, w[r][0], o);
-                const float v = fmaf(wt, is[r], z[r]);
-                const float c = fminf(fmaxf(rintf(v), 0.f), fmaxq);
-                const float wq = s[r] * (c - z[r]);
-                const float e = (wt - wq) * ut;
-                if (lane == o) {
-                    cvc[r] = c;
-                    evc[r] = e;
-                }
-                if (lane > o) w[r][0] = fmaf(-e, urow[0], w[r][0]);
-#pragma unroll
-                for (int sl = 1; sl < NSLOT; ++sl)
-                    if (q + sl < NSLOT) w[r][sl] = fmaf(-e, urow[32 * sl], w[r][sl]);
+            buf |= (unsigned long long)((cw[o >> 2] >> (8 * (o & 3))) & 0xffu) << nb;
+            nb += bits;
+            if (nb >= 32) {
+                dst[wi++] = (uint32_t)buf;
+                buf >>= 32;
+                nb -= 32;
             }
         }
-        // slot q is final: its errors (for the lazy update), codes and loss share
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            const int row = row0 + r;
-            if (rv[r]) {
-                const float eh = tcg::to_tf32(evc[r]);
-                a.err[(long long)row * a.lde + 32 * q + lane] = eh;
-                a.err_lo[(long long)row * a.lde + 32 * q + lane] = tcg::to_tf32(evc[r] - eh);
-            }
-            cb[r * B + 32 * q + lane] = (uint8_t)(int)cvc[r];
-            lacc[r] += (double)evc[r] * (double)evc[r];
-#pragma unroll
-            for (int sl = 0; sl + 1 < NSLOT; ++sl) w[r][sl] = w[r][sl + 1];
-            w[r][NSLOT - 1] = 0.f;
-        }
-    }
-    if (a.loss) {
-#pragma unroll
-        for (int r = 0; r < ROWS; ++r) {
-            const int row = row0 + r;
-            const double l = warp_sum_d(lacc[r]);
-            if (lane == 0 && rv[r]) {
-                if (j0 == 0) a.loss[row] = l;
-                else a.loss[row] += l;
-            }
-        }
-    }
-    __syncwarp();
-    const int bits = a.bits;
-    const int wpp = B * bits / 32;  // words per row for this panel
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        const int row = row0 + r;
-        if (!rv[r] || lane >= wpp) continue;
-        const int bit0 = lane * 32;
-        const int cfirst = bit0 / bits, clast = min(B - 1, (bit0 + 31) / bits);
-        uint32_t word = 0;
-        for (int c = cfirst; c <= clast; ++c) {
-            const int pos = c * bits - bit0;
-            const uint32_t code = cb[r * B + c];
-            word |= pos >= 0 ? (code << pos) : (code >> (-pos));
-        }
-        a.codes[(long long)row * a.ldcodes + (long long)j0 * bits / 32 + lane] = word;
     }
 }
 
-constexpr int COLLOOP_ROWS = 2;
-constexpr int COLLOOP_THREADS = 256;
+// Grids of groups that span several panels (group length > B), computed at the group's first
+// panel from the weights of the whole group as they stand then: one warp per row.
+__global__ void group_grid_kernel(const float *Wc, long long ldw, int m, int c0, int c1, int bits,
+                                  float *scales, uint8_t *zeros, int G, int g) {
+    const int lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (row >= m) return;
+    const float *src = Wc + (long long)row * ldw;
+    float mn = INFINITY, mx = -INFINITY;
+    for (int c = c0 + lane; c < c1; c += 32) {
+        const float x = src[c];
+        mn = fminf(mn, x);
+        mx = fmaxf(mx, x);
+    }
+    mn = warp_min(mn);
+    mx = warp_max(mx);
+    float s, is, z;
+    grid_from_range(mn, mx, (float)((1 << bits) - 1), s, is, z);
+    if (lane == 0) {
+        scales[(long long)row * G + g] = s;
+        zeros[(long long)row * G + g] = (uint8_t)z;
+    }
+}
 
-template <int NSLOT>
+template <int B>
 inline size_t colloop_smem() {
-    constexpr int B = 32 * NSLOT;
-    return (size_t)B * B * 4 + B * 4 + (COLLOOP_THREADS / 32) * COLLOOP_ROWS * B;
+    return ((size_t)B * ColloopShape<B>::LDU + B) * 4;  // U block + 1 / U[t, t]
 }
 
-template <int NSLOT>
+template <int B>
 inline int colloop_launch(const ColloopArgs &a, cudaStream_t s) {
-    const size_t smem = colloop_smem<NSLOT>();
-    GPTQ_SMEM_LIMIT((colloop_kernel<NSLOT, COLLOOP_ROWS>), smem);
-    const int rows_per_cta = (COLLOOP_THREADS / 32) * COLLOOP_ROWS;
-    colloop_kernel<NSLOT, COLLOOP_ROWS>
-        <<<ceil_div(a.m, rows_per_cta), COLLOOP_THREADS, smem, s>>>(a);
+    if (a.gs > B && a.j0 % a.gs == 0) {
+        const int c1 = a.j0 + a.gs < a.n ? a.j0 + a.gs : a.n;
+        group_grid_kernel<<<ceil_div(a.m, 8), 256, 0, s>>>(a.Wc, a.ldw, a.m, a.j0, c1, a.bits,
+                                                           a.scales, a.zeros, a.G, a.j0 / a.gs);
+        if (int st = launch_status()) return st;
+    }
+    const size_t smem = colloop_smem<B>();
+    const int rows_per_cta = COLLOOP_THREADS / ColloopShape<B>::LPR;
+    const dim3 grid(ceil_div(a.m, rows_per_cta));
+    if (a.gs < ColloopShape<B>::CPL) {
+        GPTQ_SMEM_LIMIT((colloop_kernel<B, true>), smem);
+        colloop_kernel<B, true><<<grid, COLLOOP_THREADS, smem, s>>>(a);
+    } else {
+        GPTQ_SMEM_LIMIT((colloop_kernel<B, false>), smem);
+        colloop_kernel<B, false><<<grid, COLLOOP_THREADS, smem, s>>>(a);
+    }
     return launch_status();
 }
 
@@ -322,7 +462,6 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
     ColloopArgs a;
     a.Wc = Wc; a.ldw = ldw; a.U = U; a.ldu = ldu; a.m = m; a.n = n;
     a.bits = bits; a.gs = gs;
-    a.codes = codes; a.ldcodes = (long long)n * bits / 32;
     a.scales = scales; a.zeros = zeros; a.G = group_size ? n / group_size : 1;
     a.lde = OB; a.loss = loss;
     for (int o0 = 0; o0 < n; o0 += OB) {
@@ -333,9 +472,9 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
             a.err_lo = Err_lo + (j0 - o0);
             int st;
             switch (B) {
-                case 32: st = colloop_launch<1>(a, s); break;
-                case 64: st = colloop_launch<2>(a, s); break;
-                default: st = colloop_launch<4>(a, s); break;
+                case 32: st = colloop_launch<32>(a, s); break;
+                case 64: st = colloop_launch<64>(a, s); break;
+                default: st = colloop_launch<128>(a, s); break;
             }
             if (st) return st;
             const int j1 = j0 + B;
@@ -357,7 +496,9 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
             if (int st2 = gemm_f32(p, s)) return st2;
         }
     }
-    return GPTQ_OK;
+    pack_sweep_codes_kernel<<<4 * device_sm_count(), 256, 0, s>>>(Wc, ldw, m, n, bits, COLLOOP_CPL,
+                                                                  codes, (long long)n * bits / 32);
+    return launch_status();
 }
 
 }  // namespace gptq

@@ -27,8 +27,8 @@ struct GemmArgs {
     int b_lower;        // B(k,j) = 0 for k < j
     int max_ctas;       // > 0: at most this many persistent CTAs (tensor-core path only), so
                         // that kernels on other streams keep SMs
-    int pdl;            // SIMT path: launch as a programmatic dependent of the stream's previous
-                        // kernel (the launch overlaps that kernel's tail)
+    int pdl;            // launch as a programmatic dependent of the stream's previous kernel
+                        // (the launch and the setup overlap that kernel's tail)
     const int *skip;    // when set and *skip != 0 the launch does nothing
     const float *a_lo;  // A given as tf32 hi (A) and lo (a_lo, same layout): op(A) = A + a_lo
 };

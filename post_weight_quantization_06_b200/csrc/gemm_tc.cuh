@@ -213,7 +213,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap alomap,
                TcGemmParams p) {
-    if (p.skip && *p.skip) return;   // before any barrier, TMEM or copy: every thread leaves
+    pdl_launch_next();  // the stream's next kernel may set itself up meanwhile
+    if (p.skip) {       // before any barrier, TMEM or copy: every thread leaves
+        pdl_wait_prev();
+        if (*p.skip) return;
+    }
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char *base = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
@@ -254,6 +258,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_wait_prev();  // the operands and C are the previous kernel's output from here on
 
     if (warp == 0) {
         if (lane == 0) {
@@ -603,8 +608,8 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.max_ctas > 0 && grid > g.max_ctas) grid = g.max_ctas;
     GPTQ_SMEM_LIMIT(tcg::gemm_tc_kernel, tcg::SMEM_BYTES);
     KtSpan span(s, g.skip != nullptr);
-    tcg::gemm_tc_kernel<<<grid, tcg::THREADS, tcg::SMEM_BYTES, s>>>(am, bm, cm, alm, p);
-    const int st = launch_status();
+    const int st = launch_kernel(tcg::gemm_tc_kernel, dim3(grid), dim3(tcg::THREADS), tcg::SMEM_BYTES,
+                                 s, g.pdl != 0, am, bm, cm, alm, p);
     span.done(KT_TC, g);
     return st;
 }

@@ -47,6 +47,8 @@ struct ColloopArgs {
     float *err_lo;      // tf32 pair hi = tf32(e) (err), lo = tf32(e - hi) (err_lo) that the
     long long lde;      // lazy update's tensor-core product takes without converting them
     double *loss;       // m or nullptr
+    int pdl;            // launched as a programmatic dependent (its U block loads before the
+                        // previous kernel of the stream has finished; U is not written there)
 };
 
 // Grid of one group from its range: s = (xmax - xmin)/maxq, z = rint(-xmin/s) in [0, maxq].
@@ -99,6 +101,7 @@ __global__ __launch_bounds__(COLLOOP_THREADS, 1) void colloop_kernel(ColloopArgs
     const int row = (blockIdx.x * nwarps + warp) * RPW + lane / LPR;
     const bool rv = row < a.m;
     const int j0 = a.j0;
+    pdl_launch_next();
     // U block: slot q's rows (CPL q .. CPL q + CPL-1) hold zeros left of column CPL q; from there on
     // cp.async when the rows are 16-byte aligned, else plain loads
     for (int q = 1; q < LPR; ++q) {
@@ -137,6 +140,8 @@ __global__ __launch_bounds__(COLLOOP_THREADS, 1) void colloop_kernel(ColloopArgs
             for (int c = 0; c < B; c += 32) asm volatile("prefetch.global.L2 [%0];" ::"l"(p + c));
         }
     }
+
+    pdl_wait_prev();  // the weights (and grids) are the previous kernel's output
 
     float w[CPL];
     {
@@ -415,12 +420,12 @@ inline int colloop_launch(const ColloopArgs &a, cudaStream_t s) {
     const dim3 grid(ceil_div(a.m, rows_per_cta));
     if (a.gs < ColloopShape<B>::CPL) {
         GPTQ_SMEM_LIMIT((colloop_kernel<B, true>), smem);
-        colloop_kernel<B, true><<<grid, COLLOOP_THREADS, smem, s>>>(a);
-    } else {
-        GPTQ_SMEM_LIMIT((colloop_kernel<B, false>), smem);
-        colloop_kernel<B, false><<<grid, COLLOOP_THREADS, smem, s>>>(a);
+        return launch_kernel(colloop_kernel<B, true>, grid, dim3(COLLOOP_THREADS), smem, s,
+                             a.pdl != 0, a);
     }
-    return launch_status();
+    GPTQ_SMEM_LIMIT((colloop_kernel<B, false>), smem);
+    return launch_kernel(colloop_kernel<B, false>, grid, dim3(COLLOOP_THREADS), smem, s,
+                         a.pdl != 0, a);
 }
 
 // R[t, i] = Wc[i, n + t]: the extra columns, transposed to r x m.
@@ -468,6 +473,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
         const int o1 = o0 + OB < n ? o0 + OB : n;
         for (int j0 = o0; j0 < o1; j0 += B) {
             a.j0 = j0;
+            a.pdl = j0 > 0;  // the first panel's predecessor may still be writing U
             a.err = Err + (j0 - o0);
             a.err_lo = Err_lo + (j0 - o0);
             int st;
@@ -484,6 +490,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
                                                  U + (long long)j0 * ldu + j1, ldu, 0, Wc + j1,
                                                  ldw, -1.f, 1.f);
                 p.a_lo = Err_lo + (j0 - o0);
+                p.pdl = 1;
                 if (int st2 = gemm_f32(p, s)) return st2;
             }
         }
@@ -493,6 +500,7 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
                                              U + (long long)o0 * ldu + o1, ldu, 0, Wc + o1, ldw,
                                              -1.f, 1.f);
             p.a_lo = Err_lo;
+            p.pdl = 1;
             if (int st2 = gemm_f32(p, s)) return st2;
         }
     }

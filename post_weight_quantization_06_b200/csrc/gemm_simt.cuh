@@ -31,6 +31,9 @@ struct GemmArgs {
                         // (the launch and the setup overlap that kernel's tail)
     const int *skip;    // when set and *skip != 0 the launch does nothing
     const float *a_lo;  // A given as tf32 hi (A) and lo (a_lo, same layout): op(A) = A + a_lo
+    const float *b_lo;  // B likewise: op(B) = B + b_lo (tensor-core and fp32 paths only)
+    const float *b_full;  // with b_lo: the unsplit B (row stride ldb_full), which the SIMT
+    long long ldb_full;   // path takes instead of the two parts
 };
 
 namespace simt {
@@ -193,6 +196,9 @@ inline GemmArgs<TA, TB> gemm_args(int M, int N, int K, const TA *A, long long ld
     p.pdl = 0;
     p.skip = nullptr;
     p.a_lo = nullptr;
+    p.b_lo = nullptr;
+    p.b_full = nullptr;
+    p.ldb_full = 0;
     return p;
 }
 

@@ -141,6 +141,8 @@ struct TcGemmParams {
                         // tensor add-reduction instead of a read-modify-write
     const int *skip;    // when set and *skip != 0 the launch does nothing
     int a_split;        // 1: A comes split (amap: tf32 hi, alomap: lo); only B is converted
+    int b_split;        // 1: B comes split (bmap: tf32 hi, blomap: lo); with a_split as well
+                        // nothing is converted and the MMA takes the slices as they land
 };
 
 // Bulk tensor writes of one 32 x 32 slice from shared memory (128-byte swizzle) through the C
@@ -212,7 +214,7 @@ __device__ __forceinline__ void epi_load_c(const TcGemmParams &p, int row_base, 
 __global__ void __launch_bounds__(THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap alomap,
-               TcGemmParams p) {
+               const __grid_constant__ CUtensorMap blomap, TcGemmParams p) {
     pdl_launch_next();  // the stream's next kernel may set itself up meanwhile
     if (p.skip) {       // before any barrier, TMEM or copy: every thread leaves
         pdl_wait_prev();
@@ -234,12 +236,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = num_tiles(p);
+    const bool no_conv = p.a_split && p.b_split;  // both operands arrive split
     if (threadIdx.x == 0) {
         // the descriptors' first fetch overlaps the setup instead of the first TMA load
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&amap)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&bmap)) : "memory");
         if (p.c_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&cmap)) : "memory");
         if (p.a_split) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&alomap)) : "memory");
+        if (p.b_split) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&blomap)) : "memory");
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&conv[s], CONV_WARPS);
@@ -277,7 +281,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                         break;
                     }
                     unsigned char *st = base + slot * STAGE_BYTES;
-                    mbar_expect_tx(&full[slot], (p.a_split ? 3 : 2) * SLICE_BYTES);
+                    mbar_expect_tx(&full[slot], (2 + p.a_split + p.b_split) * SLICE_BYTES);
                     if (p.a_mn) {
                         for (int q = 0; q < 4; ++q)
                             tma_load_2d(&amap, &full[slot], st + q * (BK * 128), ti * TILE + 32 * q, k0);
@@ -293,8 +297,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                     if (p.b_mn) {
                         for (int q = 0; q < 4; ++q)
                             tma_load_2d(&bmap, &full[slot], sb + q * (BK * 128), tj * TILE + 32 * q, k0);
+                        if (p.b_split)
+                            for (int q = 0; q < 4; ++q)
+                                tma_load_2d(&blomap, &full[slot], sb + SLICE_BYTES + q * (BK * 128),
+                                            tj * TILE + 32 * q, k0);
                     } else {
                         tma_load_2d(&bmap, &full[slot], sb, k0, tj * TILE);
+                        if (p.b_split) tma_load_2d(&blomap, &full[slot], sb + SLICE_BYTES, k0, tj * TILE);
                     }
                 }
             }
@@ -322,7 +331,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 const uint32_t dt = tmem + (uint32_t)(b * TILE);
                 for (int k0 = kb; k0 < ke; k0 += BK, ++it) {
                     const int slot = (int)(it % STAGES);
-                    if (!mbar_wait(&conv[slot], (uint32_t)((it / STAGES) & 1), p.wait_limit)) {
+                    if (!mbar_wait(no_conv ? &full[slot] : &conv[slot], (uint32_t)((it / STAGES) & 1),
+                                   p.wait_limit)) {
                         report(GPTQ_ERR_TIMEOUT, 13);
                         *abort_flag = 1;
                         break;
@@ -356,7 +366,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         // hi / lo split of each staged slice
         const int cw = warp - 2;
         long long it = 0;
-        for (int t = blockIdx.x; t < ntiles && !*abort_flag; t += gridDim.x) {
+        for (int t = blockIdx.x; !no_conv && t < ntiles && !*abort_flag; t += gridDim.x) {
             int ti, tj;
             tile_of(p, t, ti, tj);
             int kb, ke;
@@ -372,18 +382,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 // every thread splits CONV_PER float4 of each operand (of B alone when A came
                 // split); all of its shared-memory loads go out first so that their latencies
                 // overlap
-                const int op0 = p.a_split ? 1 : 0;
+                const int op0 = p.a_split ? 1 : 0, op1 = p.b_split ? 1 : 2;
                 float4 x[2][CONV_PER];
 #pragma unroll
                 for (int op = 0; op < 2; ++op) {
-                    if (op < op0) continue;
+                    if (op < op0 || op >= op1) continue;
                     const float4 *hi = reinterpret_cast<const float4 *>(st + op * 2 * SLICE_BYTES);
 #pragma unroll
                     for (int u = 0; u < CONV_PER; ++u) x[op][u] = hi[cw * 32 + lane + u * CONV_WARPS * 32];
                 }
 #pragma unroll
                 for (int op = 0; op < 2; ++op) {
-                    if (op < op0) continue;
+                    if (op < op0 || op >= op1) continue;
                     float4 *hi = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES);
                     float4 *lo = reinterpret_cast<float4 *>(st + op * 2 * SLICE_BYTES + SLICE_BYTES);
 #pragma unroll
@@ -558,18 +568,34 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
     static const bool force_simt = std::getenv("GPTQ_FORCE_SIMT_GEMM") != nullptr;
     const bool small = (long long)g.M * g.N < 128LL * 256 || g.K < 64;
-    // a split A on the SIMT path: C = alpha (A_hi + A_lo) B + beta C as two products
+    // split operands on the SIMT path: C = alpha (A_hi + A_lo)(B_hi + B_lo) + beta C as one
+    // product per pair of parts
     auto simt = [&]() -> int {
-        if (!g.a_lo) return gemm_simt(g, s);
         GemmArgs<float, float> h = g;
         h.a_lo = nullptr;
-        if (int st = gemm_simt(h, s)) return st;
-        h.A = g.a_lo;
-        h.beta = 1.f;
-        return gemm_simt(h, s);
+        h.b_lo = nullptr;
+        if (g.b_lo && g.b_full) {
+            h.B = g.b_full;
+            h.ldb = g.ldb_full;
+        }
+        if (!g.a_lo && (!g.b_lo || g.b_full)) return gemm_simt(h, s);
+        const float *as[2] = {g.A, g.a_lo}, *bs[2] = {h.B, g.b_full ? nullptr : g.b_lo};
+        bool first = true;
+        for (int i = 0; i < 2; ++i) {
+            for (int j = 0; j < 2; ++j) {
+                if (!as[i] || !bs[j]) continue;
+                h.A = as[i];
+                h.B = bs[j];
+                h.beta = first ? g.beta : 1.f;
+                first = false;
+                if (int st = gemm_simt(h, s)) return st;
+            }
+        }
+        return GPTQ_OK;
     };
     if (small || !tcg::tc_eligible(g.A, g.lda, g.B, g.ldb) ||
         (g.a_lo && !tcg::tc_eligible(g.a_lo, g.lda, g.B, g.ldb)) ||
+        (g.b_lo && !tcg::tc_eligible(g.A, g.lda, g.b_lo, g.ldb)) ||
         (reinterpret_cast<uintptr_t>(g.C) & 3u) || force_simt)
         return simt();
     tcg::TcGemmParams p;
@@ -582,7 +608,8 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     p.b_upper = g.b_upper; p.b_lower = g.b_lower;
     p.tiles_m = ceil_div(g.M, tcg::TILE);
     p.tiles_n = ceil_div(g.N, tcg::TILE);
-    p.wait_limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
+    static const long long wait_limit = tc::env_ll("GPTQ_WAIT_LIMIT_CYCLES", 4000000000LL);
+    p.wait_limit = wait_limit;
     p.skip = g.skip;
     CUtensorMap am, bm, cm;
     const bool ok_a = p.a_mn ? tcg::make_map_f32(&am, g.A, g.K, g.M, g.lda, 32, 32, true)
@@ -594,8 +621,14 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     const bool ok_al = !g.a_lo ||
         (p.a_mn ? tcg::make_map_f32(&alm, g.a_lo, g.K, g.M, g.lda, 32, 32, true)
                 : tcg::make_map_f32(&alm, g.a_lo, g.M, g.K, g.lda, 32, tcg::TILE, false));
-    if (!ok_a || !ok_b || !ok_al) return simt();
+    CUtensorMap blm;
+    p.b_split = g.b_lo ? 1 : 0;
+    const bool ok_bl = !g.b_lo ||
+        (p.b_mn ? tcg::make_map_f32(&blm, g.b_lo, g.K, g.N, g.ldb, 32, 32, true)
+                : tcg::make_map_f32(&blm, g.b_lo, g.N, g.K, g.ldb, 32, tcg::TILE, false));
+    if (!ok_a || !ok_b || !ok_al || !ok_bl) return simt();
     if (!g.a_lo) alm = am;   // not read
+    if (!g.b_lo) blm = bm;   // not read
     // C through a tensor map when beta is 0 or 1 and C's base and pitch allow it
     static const bool rmw_only = std::getenv("GPTQ_GEMM_RMW_EPILOGUE") != nullptr;
     p.c_tma = !rmw_only && (g.beta == 0.f || g.beta == 1.f) &&
@@ -609,7 +642,7 @@ inline int gemm_f32(const GemmArgs<float, float> &g, cudaStream_t s) {
     GPTQ_SMEM_LIMIT(tcg::gemm_tc_kernel, tcg::SMEM_BYTES);
     KtSpan span(s, g.skip != nullptr);
     const int st = launch_kernel(tcg::gemm_tc_kernel, dim3(grid), dim3(tcg::THREADS), tcg::SMEM_BYTES,
-                                 s, g.pdl != 0, am, bm, cm, alm, p);
+                                 s, g.pdl != 0, am, bm, cm, alm, blm, p);
     span.done(KT_TC, g);
     return st;
 }

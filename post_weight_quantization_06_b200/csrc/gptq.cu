@@ -43,16 +43,21 @@ inline FactorWs carve_factor(Carver &c, long long n) {
 }
 
 struct QuantWs {
-    float *Wc, *Err, *Err_lo;
+    float *Wc, *Err, *Err_lo, *Uh, *Ul;
 };
 // Err holds the errors of one outer block of the two-level lazy update: m x OB with
-// OB <= min(QUANT_OUTER_MAX, n).
-inline QuantWs carve_quant(Carver &c, long long m, long long N, int B) {
+// OB <= min(QUANT_OUTER_MAX, n). With `band`, Uh / Ul hold one outer block's rows of U split
+// into tf32 pairs (OB x N each), so that the lazy updates convert nothing; without it (the
+// no-allocation entry point's fixed scratch) they are null and the updates split U as they go.
+inline QuantWs carve_quant(Carver &c, long long m, long long N, int B, bool band = true) {
     QuantWs w;
     w.Wc = c.take<float>((size_t)m * N);
-    const long long ob = N < QUANT_OUTER_MAX ? N : QUANT_OUTER_MAX;
-    w.Err = c.take<float>((size_t)m * (ob > B ? ob : B));
-    w.Err_lo = c.take<float>((size_t)m * (ob > B ? ob : B));
+    const long long ob0 = N < QUANT_OUTER_MAX ? N : QUANT_OUTER_MAX;
+    const long long ob = ob0 > B ? ob0 : B;
+    w.Err = c.take<float>((size_t)m * ob);
+    w.Err_lo = c.take<float>((size_t)m * ob);
+    w.Uh = band ? c.take<float>((size_t)ob * N) : nullptr;
+    w.Ul = band ? c.take<float>((size_t)ob * N) : nullptr;
     return w;
 }
 
@@ -451,7 +456,7 @@ static int gptq_quantize_layer_body(const void *W, int w_dtype, int64_t m, int64
     QuantWs w = carve_quant(c, m, n, block_size);
     if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
     return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
-                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, s);
+                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, w.Uh, w.Ul, s);
 }
 
 GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t n, const float *U,
@@ -471,18 +476,19 @@ static int gptq_quantize_layer_noalloc_body(const void *W, int w_dtype, int64_t 
     if (!W || !U || !codes || !scales || !zeros) return GPTQ_ERR_ARG;
     if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_ARG;
     if (!valid_quant_args(m, n, bits, group_size, block_size)) return GPTQ_ERR_ARG;
-    const size_t need = gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size);
-    if (need > GPTQ_NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
+    Carver sz(nullptr);
+    carve_quant(sz, m, n, block_size, false);
+    if (sz.off > GPTQ_NOALLOC_SCRATCH_BYTES) return GPTQ_ERR_ARG;
     void *scratch = noalloc_scratch();
     if (!scratch) return GPTQ_ERR_CUDA;
     // The working copy and the per-panel errors are fully written before they are read, so
     // nothing left in the shared scratch by an earlier call needs clearing.
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     Carver c(scratch);
-    QuantWs w = carve_quant(c, m, n, block_size);
+    QuantWs w = carve_quant(c, m, n, block_size, false);
     if (int st = init_work(W, w_dtype, m, (int)n, w.Wc, n, (int)n, s)) return st;
     return sweep_layer(w.Wc, n, (int)m, (int)n, (int)n, U, n, bits, group_size, block_size,
-                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, s);
+                       codes, scales, zeros, loss_out, w.Err, w.Err_lo, nullptr, nullptr, s);
 }
 
 GPTQ_API int gptq_quantize_layer_noalloc(const void *W, int w_dtype, int64_t m, int64_t n,
@@ -523,7 +529,8 @@ static int gptq_il_quantize_layer_body(const void *W, int w_dtype, int64_t m, in
     }
     if (int st = init_work(W, w_dtype, m, (int)n, w.q.Wc, N, (int)N, s)) return st;
     if (int st = sweep_layer(w.q.Wc, N, (int)m, (int)n, (int)N, w.Uaug, N, bits, group_size,
-                             block_size, codes, scales, zeros, loss_out, w.q.Err, w.q.Err_lo, s))
+                             block_size, codes, scales, zeros, loss_out, w.q.Err, w.q.Err_lo,
+                             w.q.Uh, w.q.Ul, s))
         return st;
     if (r > 0) {
         extract_R_kernel<<<592, 256, 0, s>>>(w.q.Wc, N, (int)m, (int)n, r, R);

@@ -438,6 +438,27 @@ __global__ void extract_R_kernel(const float *Wc, long long ldw, int m, int n, i
     }
 }
 
+// Rows r0 .. r1-1 of U, columns c0 .. N-1, split into tf32 pairs (round to nearest, as the
+// tensor-core product's converters would): Uh[i, c] = tf32(U[r0 + i, c]),
+// Ul[i, c] = tf32(U[r0 + i, c] - Uh[i, c]) (row stride N).
+__global__ void split_band_kernel(const float *U, long long ldu, int r0, int r1, int c0, int N,
+                                  float *Uh, float *Ul) {
+    const int w4 = (N - c0) / 4;  // c0 and N are multiples of 4
+    const long long total = (long long)(r1 - r0) * w4;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int i = (int)(idx / w4), c = c0 + 4 * (int)(idx % w4);
+        const float4 v = *reinterpret_cast<const float4 *>(U + (long long)(r0 + i) * ldu + c);
+        float4 h, l;
+        h.x = tcg::to_tf32(v.x); l.x = tcg::to_tf32(v.x - h.x);
+        h.y = tcg::to_tf32(v.y); l.y = tcg::to_tf32(v.y - h.y);
+        h.z = tcg::to_tf32(v.z); l.z = tcg::to_tf32(v.z - h.z);
+        h.w = tcg::to_tf32(v.w); l.w = tcg::to_tf32(v.w - h.w);
+        *reinterpret_cast<float4 *>(Uh + (long long)i * N + c) = h;
+        *reinterpret_cast<float4 *>(Ul + (long long)i * N + c) = l;
+    }
+}
+
 // The sweep over all panels of a prepared working copy Wc (m x N, first n columns quantized).
 // Width of the outer blocks of the two-level lazy update: 1024 columns (or n if smaller) when
 // every group that starts inside an outer block also ends inside it, i.e. for one group per
@@ -460,7 +481,7 @@ inline int outer_block(int n, int gs, int B) {
 inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const float *U,
                        long long ldu, int bits, int group_size, int B, uint32_t *codes,
                        float *scales, uint8_t *zeros, double *loss, float *Err, float *Err_lo,
-                       cudaStream_t s) {
+                       float *Uh, float *Ul, cudaStream_t s) {
     KtStageScope stage(GPTQ_KT_SWEEP);
     const int gs = group_size ? group_size : n;
     const int OB = outer_block(n, gs, B);
@@ -469,8 +490,20 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
     a.bits = bits; a.gs = gs;
     a.scales = scales; a.zeros = zeros; a.G = group_size ? n / group_size : 1;
     a.lde = OB; a.loss = loss;
+    // the band of U that an outer block's updates read, split once (when U's rows allow
+    // 16-byte vectors and the caller gave room for it)
+    const bool band = Uh && Ul && ldu % 4 == 0 && N % 4 == 0 &&
+                      ((reinterpret_cast<uintptr_t>(U) | reinterpret_cast<uintptr_t>(Uh) |
+                        reinterpret_cast<uintptr_t>(Ul)) & 15u) == 0;
     for (int o0 = 0; o0 < n; o0 += OB) {
         const int o1 = o0 + OB < n ? o0 + OB : n;
+        if (band) {
+            split_band_kernel<<<4 * device_sm_count(), 256, 0, s>>>(U, ldu, o0, o1, o0, N, Uh, Ul);
+            if (int st = launch_status()) return st;
+        }
+        // B operand of an update reading U[j, c] (j in this outer block): the band's pair
+        auto bh = [&](int j, int c) { return Uh + (long long)(j - o0) * N + c; };
+        auto bl = [&](int j, int c) { return Ul + (long long)(j - o0) * N + c; };
         for (int j0 = o0; j0 < o1; j0 += B) {
             a.j0 = j0;
             a.pdl = j0 > 0;  // the first panel's predecessor may still be writing U
@@ -486,20 +519,34 @@ inline int sweep_layer(float *Wc, long long ldw, int m, int n, int N, const floa
             const int j1 = j0 + B;
             if (j1 < o1) {
                 // inner: Wc[:, j1:o1] -= Err_panel (m x B) * U[j0:j1, j1:o1]
-                auto p = gemm_args<float, float>(m, o1 - j1, B, Err + (j0 - o0), OB, 0,
-                                                 U + (long long)j0 * ldu + j1, ldu, 0, Wc + j1,
-                                                 ldw, -1.f, 1.f);
+                auto p = band ? gemm_args<float, float>(m, o1 - j1, B, Err + (j0 - o0), OB, 0,
+                                                        bh(j0, j1), N, 0, Wc + j1, ldw, -1.f, 1.f)
+                              : gemm_args<float, float>(m, o1 - j1, B, Err + (j0 - o0), OB, 0,
+                                                        U + (long long)j0 * ldu + j1, ldu, 0,
+                                                        Wc + j1, ldw, -1.f, 1.f);
                 p.a_lo = Err_lo + (j0 - o0);
+                if (band) {
+                    p.b_lo = bl(j0, j1);
+                    p.b_full = U + (long long)j0 * ldu + j1;
+                    p.ldb_full = ldu;
+                }
                 p.pdl = 1;
                 if (int st2 = gemm_f32(p, s)) return st2;
             }
         }
         if (o1 < N) {
             // outer: Wc[:, o1:N] -= Err_outer (m x (o1 - o0)) * U[o0:o1, o1:N]
-            auto p = gemm_args<float, float>(m, N - o1, o1 - o0, Err, OB, 0,
-                                             U + (long long)o0 * ldu + o1, ldu, 0, Wc + o1, ldw,
-                                             -1.f, 1.f);
+            auto p = band ? gemm_args<float, float>(m, N - o1, o1 - o0, Err, OB, 0, bh(o0, o1), N,
+                                                    0, Wc + o1, ldw, -1.f, 1.f)
+                          : gemm_args<float, float>(m, N - o1, o1 - o0, Err, OB, 0,
+                                                    U + (long long)o0 * ldu + o1, ldu, 0, Wc + o1,
+                                                    ldw, -1.f, 1.f);
             p.a_lo = Err_lo;
+            if (band) {
+                p.b_lo = bl(o0, o1);
+                p.b_full = U + (long long)o0 * ldu + o1;
+                p.ldb_full = ldu;
+            }
             p.pdl = 1;
             if (int st2 = gemm_f32(p, s)) return st2;
         }

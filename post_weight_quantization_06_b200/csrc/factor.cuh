@@ -210,6 +210,8 @@ constexpr int LB_TLD = FACTOR_NB - LB + 4;
 constexpr int LEAF_THREADS = 256;
 constexpr size_t LEAF_BLK_SMEM =
     sizeof(float) * (2 * (size_t)FACTOR_NB * LB_LD + (size_t)LB * LB_TLD + 2 * LB);
+constexpr size_t LEAF_EXCLUSIVE_SMEM = 227 * 1024;  // the per-block maximum on sm_100
+static_assert(LEAF_BLK_SMEM <= LEAF_EXCLUSIVE_SMEM, "leaf fits the exclusive allocation");
 
 // A: X_kk of the 32 x 32 block of S at (r, r), written to X (warp 0 only). Before step c,
 // physical register p holds column (p - 31 + c) mod 32, so the pivot is always m[31]; the
@@ -436,18 +438,24 @@ inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, i
     // GPTQ_LEAF=0 selects the barrier-synchronised leaf (diag_ul_inv_kernel)
     static const bool blocked = tc::env_ll("GPTQ_LEAF", 1) != 0;
     if (!blocked) return diag_ul_inv<float>(A, lda, U, ldu, nb, col_base, s);
-    GPTQ_SMEM_LIMIT(leaf_blk_kernel, LEAF_BLK_SMEM);
-    return launch_kernel(leaf_blk_kernel, dim3(1), dim3(LEAF_THREADS), LEAF_BLK_SMEM, s, pdl, A,
+    // With GPTQ_LEAF_EXCLUSIVE (default 1) the leaf asks for the whole of its SM's shared
+    // memory, so that no CTA of the concurrent GEMMs lands beside it and takes its issue slots.
+    static const bool exclusive = tc::env_ll("GPTQ_LEAF_EXCLUSIVE", 1) != 0;
+    const size_t smem = exclusive ? LEAF_EXCLUSIVE_SMEM : LEAF_BLK_SMEM;
+    GPTQ_SMEM_LIMIT(leaf_blk_kernel, smem);
+    return launch_kernel(leaf_blk_kernel, dim3(1), dim3(LEAF_THREADS), smem, s, pdl, A,
                          lda, U, ldu, nb, col_base);
 }
 
-// Streams of the blocked factor: the pivot chain (leaf, panel solve, look-ahead column) on a
-// high-priority stream, the trailing update and the inverse's rows on two others. One set per
-// device, made on the first call; the mutex keeps the event protocol of one call intact
-// against calls from other host threads.
+// Streams of the blocked factor: the pivot chain (leaf, and the two 128 x 128 products that
+// feed the next leaf) on a high-priority stream; the rest of each panel and look-ahead column,
+// the trailing update and the inverse's rows on three others. One set per device and slot,
+// made on the first call; the mutex keeps the event protocol of one call intact against calls
+// from other host threads.
 struct FactorStreams {
-    cudaStream_t chain = nullptr, bulk = nullptr, inv = nullptr;
-    cudaEvent_t fork = nullptr, panel = nullptr, bulk_done = nullptr, join[3] = {};
+    cudaStream_t chain = nullptr, panel = nullptr, bulk = nullptr, inv = nullptr;
+    cudaEvent_t fork = nullptr, leaf_done = nullptr, pdiag_done = nullptr, prest_done = nullptr,
+                larest_done = nullptr, bulk_done = nullptr, join[4] = {};
     std::mutex mu;
     bool ready = false;
 };
@@ -466,9 +474,11 @@ inline FactorStreams *factor_streams(int slot) {
         int lo = 0, hi = 0;
         cudaDeviceGetStreamPriorityRange(&lo, &hi);
         bool ok = cudaStreamCreateWithPriority(&f.chain, cudaStreamNonBlocking, hi) == cudaSuccess &&
+                  cudaStreamCreateWithPriority(&f.panel, cudaStreamNonBlocking, hi) == cudaSuccess &&
                   cudaStreamCreateWithPriority(&f.bulk, cudaStreamNonBlocking, lo) == cudaSuccess &&
                   cudaStreamCreateWithPriority(&f.inv, cudaStreamNonBlocking, lo) == cudaSuccess;
-        cudaEvent_t *evs[] = {&f.fork, &f.panel, &f.bulk_done, &f.join[0], &f.join[1], &f.join[2]};
+        cudaEvent_t *evs[] = {&f.fork, &f.leaf_done, &f.pdiag_done, &f.prest_done, &f.larest_done,
+                              &f.bulk_done, &f.join[0], &f.join[1], &f.join[2], &f.join[3]};
         for (cudaEvent_t *e : evs)
             ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
         if (!ok) return nullptr;
@@ -482,15 +492,20 @@ inline FactorStreams *factor_streams(int slot) {
 // lower block rows receive the panels transposed and the upper triangle is consumed. U (n x
 // n, ldu) must be zero on entry and receives U = Ubar^-1, where A = Ubar Ubar^T, Ubar upper
 // (so that A^-1 = U^T U with U upper: the factor the column sweep uses). With 128-column
-// blocks k = K-1 .. 0, r = first column of block k:
-//   chain  X_kk  = leaf(A_kk)                              (Ubar_kk^-1)
-//          L_k^T = X_kk A[0:r, k]^T                         (panel of Ubar, kept transposed)
-//          A[0:r, k-1] -= L_k L_k[k-1]^T                    (look-ahead: the next panel)
-//   bulk   A[0:r', 0:r'] -= L_k L_k^T on r' = start of block k-1 (upper triangle)
+// blocks k = K-1 .. 0, r = first column of block k, r1 = r - 128 (block k-1):
+//   chain  X_kk  = leaf(A_kk)                                (Ubar_kk^-1)
+//          L_k[k-1]^T = X_kk A[r1:r, k]^T                     (the panel's rows of block k-1)
+//          A[r1:r, k-1] -= L_k[k-1] L_k[k-1]^T                (look-ahead: the next diagonal)
+//   panel  L_k[0:r1]^T = X_kk A[0:r1, k]^T                    (the rest of the panel)
+//          A[0:r1, k-1] -= L_k[0:r1] L_k[k-1]^T               (the rest of the look-ahead)
+//   bulk   A[0:r1, 0:r1] -= L_k[0:r1] L_k[0:r1]^T              (upper triangle)
 //   inv    U[k, >k] = -X_kk P[k, >k],  P[0:r, k:] += L_k U[k, k:]
 // where P = U's upper part before its row block is final: P[i, j] = sum_l Ubar[i, l] X[l, j]
-// over the finished row blocks l, from Ubar X = I. The chain waits for the bulk update of
-// the previous block before its look-ahead; the inverse stream trails both.
+// over the finished row blocks l, from Ubar X = I. Only the chain is serial from block to
+// block. Its products for block k-1 wait for the look-ahead rest of block k+1 (rows of block
+// k-1 in column block k) and for the trailing update of block k+1 (which also writes the next
+// diagonal block); the panel's look-ahead waits for that trailing update too (both write
+// column block k-1).
 inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, int n, float *T,
                              cudaStream_t s, int slot = 0) {
     KtStageScope stage(GPTQ_KT_FACTOR);
@@ -499,47 +514,73 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
     if (!fs) return GPTQ_ERR_CUDA;
     std::lock_guard<std::mutex> lk(fs->mu);
     const int sms = device_sm_count();
-    // persistent CTAs of each side-stream GEMM: the rest of the SMs stay free for the chain
+    // persistent CTAs of the trailing update and of the inverse's GEMMs: the rest of the SMs
+    // stay free for the chain and the panel stream
     static const long long side_env = tc::env_ll("GPTQ_FACTOR_SIDE_CTAS", 0);
+    static const long long bulk_env = tc::env_ll("GPTQ_FACTOR_BULK_CTAS", 0);
+    static const long long inv_env = tc::env_ll("GPTQ_FACTOR_INV_CTAS", 0);
     const int side = side_env > 0 ? (int)side_env : (2 * sms) / 3;
+    const int bulk_ctas = bulk_env > 0 ? (int)bulk_env : side;
+    const int inv_ctas = inv_env > 0 ? (int)inv_env : side;
     if (cudaEventRecord(fs->fork, s) != cudaSuccess) return GPTQ_ERR_CUDA;
-    cudaStreamWaitEvent(fs->chain, fs->fork, 0);
-    cudaStreamWaitEvent(fs->bulk, fs->fork, 0);
-    cudaStreamWaitEvent(fs->inv, fs->fork, 0);
+    cudaStream_t streams[4] = {fs->chain, fs->panel, fs->bulk, fs->inv};
+    for (cudaStream_t st2 : streams) cudaStreamWaitEvent(st2, fs->fork, 0);
     const int K = ceil_div(n, FACTOR_NB);
     int st = GPTQ_OK;
     for (int k = K - 1; k >= 0 && st == GPTQ_OK; --k) {
         const int r = k * FACTOR_NB, bk = std::min(FACTOR_NB, n - r);
+        const int r1 = r - FACTOR_NB;  // first column of block k-1 (k > 0)
         float *Xkk = U + (long long)r * ldu + r;
         float *Lt = A + (long long)r * lda;  // L_k^T: bk x r, strict lower block row k
-        // the chain's leaf and panel product start while their predecessors finish
+        // chain: the leaf starts while its predecessor (the last look-ahead) finishes
         if ((st = leaf_ul_inv(A + (long long)r * lda + r, lda, Xkk, ldu, bk, r, fs->chain, true))) break;
+        cudaEventRecord(fs->leaf_done, fs->chain);
         if (k > 0) {
-            auto p = gemm_args<float, float>(bk, r, bk, Xkk, ldu, 0, A + r, lda, 1, Lt, lda, 1.f, 0.f);
+            // rows of block k-1 in column block k carry the look-ahead rest of block k+1
+            if (k < K - 1) cudaStreamWaitEvent(fs->chain, fs->larest_done, 0);
+            auto p = gemm_args<float, float>(bk, FACTOR_NB, bk, Xkk, ldu, 0,
+                                             A + (long long)r1 * lda + r, lda, 1, Lt + r1, lda,
+                                             1.f, 0.f);
             p.a_upper = 1;
             p.pdl = 1;
-            // the chain's products are small (K = 128, at most 47 output tiles of 128): the SIMT
-            // kernel's 64-tiles start sooner and spread wider than the tensor-core pipeline
             if ((st = gemm_simt(p, fs->chain))) break;
+            cudaEventRecord(fs->pdiag_done, fs->chain);
+            // the next diagonal block, after the trailing update of block k+1 has written it
+            if (k < K - 1) cudaStreamWaitEvent(fs->chain, fs->bulk_done, 0);
+            auto q = gemm_args<float, float>(FACTOR_NB, FACTOR_NB, bk, Lt + r1, lda, 1, Lt + r1, lda,
+                                             0, A + (long long)r1 * lda + r1, lda, -1.f, 1.f);
+            q.pdl = 1;
+            if ((st = gemm_simt(q, fs->chain))) break;
         }
-        cudaEventRecord(fs->panel, fs->chain);
-        if (k > 0) {
-            const int r1 = r - FACTOR_NB;
-            cudaStreamWaitEvent(fs->chain, fs->bulk_done, 0);  // bulk update of block k+1
-            auto p = gemm_args<float, float>(r, FACTOR_NB, bk, Lt, lda, 1, Lt + r1, lda, 0, A + r1,
-                                             lda, -1.f, 1.f);
+        // panel: the rest of L_k and of the look-ahead column
+        if (k > 1) {
+            cudaStreamWaitEvent(fs->panel, fs->leaf_done, 0);
+            auto p = gemm_args<float, float>(bk, r1, bk, Xkk, ldu, 0, A + r, lda, 1, Lt, lda, 1.f, 0.f);
+            p.a_upper = 1;
             p.pdl = 1;
-            if ((st = gemm_simt(p, fs->chain))) break;
-            if (r1 > 0) {
-                cudaStreamWaitEvent(fs->bulk, fs->panel, 0);
-                auto q = gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);
-                q.c_upper = 1;
-                q.max_ctas = side;
-                if ((st = gemm_f32(q, fs->bulk))) break;
-                cudaEventRecord(fs->bulk_done, fs->bulk);
-            }
+            if ((st = gemm_simt(p, fs->panel))) break;
+            cudaEventRecord(fs->prest_done, fs->panel);
+            cudaStreamWaitEvent(fs->panel, fs->pdiag_done, 0);
+            if (k < K - 1) cudaStreamWaitEvent(fs->panel, fs->bulk_done, 0);
+            auto q = gemm_args<float, float>(r1, FACTOR_NB, bk, Lt, lda, 1, Lt + r1, lda, 0, A + r1,
+                                             lda, -1.f, 1.f);
+            q.pdl = 1;
+            if ((st = gemm_simt(q, fs->panel))) break;
+            cudaEventRecord(fs->larest_done, fs->panel);
+            // bulk: the trailing update of everything left of block k-1
+            cudaStreamWaitEvent(fs->bulk, fs->prest_done, 0);
+            auto b2 = gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);
+            b2.c_upper = 1;
+            b2.max_ctas = bulk_ctas;
+            if ((st = gemm_f32(b2, fs->bulk))) break;
+            cudaEventRecord(fs->bulk_done, fs->bulk);
         }
-        cudaStreamWaitEvent(fs->inv, fs->panel, 0);
+        // inverse rows: need X_kk and the whole panel L_k
+        cudaStreamWaitEvent(fs->inv, fs->leaf_done, 0);
+        if (k > 0) {
+            cudaStreamWaitEvent(fs->inv, fs->pdiag_done, 0);
+            if (k > 1) cudaStreamWaitEvent(fs->inv, fs->prest_done, 0);
+        }
         if (k < K - 1) {
             const int e = r + bk, wdt = n - e;
             float *row = U + (long long)r * ldu + e;
@@ -551,20 +592,20 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
             }
             auto p = gemm_args<float, float>(bk, wdt, bk, Xkk, ldu, 0, T, wdt, 0, row, ldu, -1.f, 0.f);
             p.a_upper = 1;
-            p.max_ctas = side;
+            p.max_ctas = inv_ctas;
             if ((st = gemm_f32(p, fs->inv))) break;
         }
         if (k > 0) {
             auto p = gemm_args<float, float>(r, n - r, bk, Lt, lda, 1, Xkk, ldu, 0, U + r, ldu, 1.f, 1.f);
-            p.max_ctas = side;
+            p.max_ctas = inv_ctas;
             if ((st = gemm_f32(p, fs->inv))) break;
         }
     }
-    // join all three streams back into the caller's stream, on success and on error alike
-    cudaEventRecord(fs->join[0], fs->chain);
-    cudaEventRecord(fs->join[1], fs->bulk);
-    cudaEventRecord(fs->join[2], fs->inv);
-    for (int i = 0; i < 3; ++i) cudaStreamWaitEvent(s, fs->join[i], 0);
+    // join all four streams back into the caller's stream, on success and on error alike
+    for (int i = 0; i < 4; ++i) {
+        cudaEventRecord(fs->join[i], streams[i]);
+        cudaStreamWaitEvent(s, fs->join[i], 0);
+    }
     if (st == GPTQ_OK && cudaGetLastError() != cudaSuccess) st = GPTQ_ERR_CUDA;
     return st;
 }

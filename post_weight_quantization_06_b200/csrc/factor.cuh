@@ -447,6 +447,25 @@ inline int leaf_ul_inv(const float *A, long long lda, float *U, long long ldu, i
                          lda, U, ldu, nb, col_base);
 }
 
+// Scratch of factor_ul_inverse, in blocks of FACTOR_NB x n floats: a copy of one row block of
+// U, and the panel split into tf32 pairs for the trailing update.
+constexpr int FACTOR_T_BLOCKS = 3;
+
+// Lt[:, 0:cols] (rows x cols, row stride lda) split into tf32 pairs (round to nearest), row
+// stride cols: the trailing update's operands, which then need no conversion.
+__global__ void split_panel_kernel(const float *Lt, long long lda, int rows, int cols, float *Lh,
+                                   float *Ll) {
+    const long long total = (long long)rows * cols;
+    for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+         idx += (long long)gridDim.x * blockDim.x) {
+        const int i = (int)(idx / cols), j = (int)(idx % cols);
+        const float v = Lt[(long long)i * lda + j];
+        const float h = tcg::to_tf32(v);
+        Lh[idx] = h;
+        Ll[idx] = tcg::to_tf32(v - h);
+    }
+}
+
 // Streams of the blocked factor: the pivot chain (leaf, and the two 128 x 128 products that
 // feed the next leaf) on a high-priority stream; the rest of each panel and look-ahead column,
 // the trailing update and the inverse's rows on three others. One set per device and slot,
@@ -492,7 +511,8 @@ inline FactorStreams *factor_streams(int slot) {
 // lower block rows receive the panels transposed and the upper triangle is consumed. U (n x
 // n, ldu) must be zero on entry and receives U = Ubar^-1, where A = Ubar Ubar^T, Ubar upper
 // (so that A^-1 = U^T U with U upper: the factor the column sweep uses). With 128-column
-// blocks k = K-1 .. 0, r = first column of block k, r1 = r - 128 (block k-1):
+// blocks k = K-1 .. 0, r = first column of block k, r1 = r - 128 (block k-1). T holds
+// FACTOR_T_BLOCKS x 128 x n floats of scratch.
 //   chain  X_kk  = leaf(A_kk)                                (Ubar_kk^-1)
 //          L_k[k-1]^T = X_kk A[r1:r, k]^T                     (the panel's rows of block k-1)
 //          A[r1:r, k-1] -= L_k[k-1] L_k[k-1]^T                (look-ahead: the next diagonal)
@@ -567,9 +587,23 @@ inline int factor_ul_inverse(float *A, long long lda, float *U, long long ldu, i
             q.pdl = 1;
             if ((st = gemm_simt(q, fs->panel))) break;
             cudaEventRecord(fs->larest_done, fs->panel);
-            // bulk: the trailing update of everything left of block k-1
+            // bulk: the trailing update of everything left of block k-1, from the panel split
+            // once into tf32 pairs (both operands are L_k)
             cudaStreamWaitEvent(fs->bulk, fs->prest_done, 0);
-            auto b2 = gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);
+            float *Lh = T + (size_t)FACTOR_NB * n, *Ll = Lh + (size_t)FACTOR_NB * n;
+            const bool split = r1 >= 256 && r1 % 4 == 0 && (reinterpret_cast<uintptr_t>(Lh) & 15u) == 0;
+            if (split) {
+                split_panel_kernel<<<2 * sms, 256, 0, fs->bulk>>>(Lt, lda, bk, r1, Lh, Ll);
+                if ((st = launch_status())) break;
+            }
+            auto b2 = split ? gemm_args<float, float>(r1, r1, bk, Lh, r1, 1, Lh, r1, 0, A, lda, -1.f, 1.f)
+                            : gemm_args<float, float>(r1, r1, bk, Lt, lda, 1, Lt, lda, 0, A, lda, -1.f, 1.f);
+            if (split) {
+                b2.a_lo = Ll;
+                b2.b_lo = Ll;
+                b2.b_full = Lt;
+                b2.ldb_full = lda;
+            }
             b2.c_upper = 1;
             b2.max_ctas = bulk_ctas;
             if ((st = gemm_f32(b2, fs->bulk))) break;

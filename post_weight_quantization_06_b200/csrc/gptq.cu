@@ -38,7 +38,7 @@ struct FactorWs {
 inline FactorWs carve_factor(Carver &c, long long n) {
     FactorWs w;
     w.A = c.take<float>((size_t)n * n);
-    w.T = c.take<float>((size_t)FACTOR_NB * n);
+    w.T = c.take<float>((size_t)FACTOR_T_BLOCKS * FACTOR_NB * n);
     return w;
 }
 

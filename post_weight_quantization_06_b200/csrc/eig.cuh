@@ -87,6 +87,8 @@ __device__ __forceinline__ double safe_pivot(double D, double pivmin) {
 __global__ __launch_bounds__(EIG_THREADS) void sym_eig_top_kernel(const double *Tin, int p, int r,
                                                                   double *evals, double *Qout,
                                                                   const int *skip) {
+    pdl_wait_prev();
+    pdl_launch_next();
     if (skip && *skip) return;
     extern __shared__ __align__(16) double esm[];
     double *Vh = esm;                              // packed Householder vectors
@@ -463,8 +465,8 @@ inline int sym_eig_top(const double *T, int p, int r, double *evals, double *Q, 
     if (p < 1 || p > EIG_MAXP || r < 1 || r > p) return GPTQ_ERR_ARG;
     const size_t smem = eig_smem(p);
     GPTQ_SMEM_LIMIT(sym_eig_top_kernel, eig_smem(EIG_MAXP));
-    sym_eig_top_kernel<<<1, EIG_THREADS, smem, s>>>(T, p, r, evals, Q, skip);
-    return launch_status();
+    return launch_kernel(sym_eig_top_kernel, dim3(1), dim3(EIG_THREADS), smem, s, true, T, p, r,
+                         evals, Q, skip);
 }
 
 }  // namespace gptq

@@ -49,6 +49,8 @@ template <typename T>
 __global__ __launch_bounds__(DiagCfg<T>::TG * DiagCfg<T>::TG) void diag_ul_inv_kernel(
     const T *A, long long lda, T *U, long long ldu, int nb, long long col_base, const int *skip) {
     constexpr int TG = DiagCfg<T>::TG, TS = DiagCfg<T>::TS;
+    pdl_wait_prev();
+    pdl_launch_next();
     if (skip && *skip) return;
     // wb[c'] = M[c'][c] for c' < c (column c), -1 at c, M[c][c'] for c' > c (row c); the
     // pivot M[c][c] separately. Then u_i = ipiv wb[i] (i < c) and v_j = -ipiv wb[j].
@@ -150,8 +152,8 @@ template <typename T>
 inline int diag_ul_inv(const T *A, long long lda, T *U, long long ldu, int nb, long long col_base,
                        cudaStream_t s, const int *skip = nullptr) {
     constexpr int TG = DiagCfg<T>::TG;
-    diag_ul_inv_kernel<T><<<1, TG * TG, 0, s>>>(A, lda, U, ldu, nb, col_base, skip);
-    return launch_status();
+    return launch_kernel(diag_ul_inv_kernel<T>, dim3(1), dim3(TG * TG), 0, s, true, A, lda, U, ldu,
+                         nb, col_base, skip);
 }
 
 // A_work = H + lambda I (full copy), lambda = lambda_rel * mean(diag H) written to *lam.

@@ -308,6 +308,8 @@ __global__ __launch_bounds__(256) void gemm_f64acc_kernel(int M, int N, int K, c
                                                           int b_upper, F64Epilogue ep,
                                                           double *part, int kchunk) {
     constexpr int T = F64_T, BK = F64_BK, PER = T * BK / 256;  // 8 elements per thread
+    pdl_wait_prev();
+    pdl_launch_next();
     if (ep.skip && *ep.skip) return;
     __shared__ double As[BK][T + 1];
     __shared__ double Bs[BK][T + 1];
@@ -399,6 +401,8 @@ template <typename TA, typename TB, typename TC>
 __global__ __launch_bounds__(256, 2) void gemm_f64acc_big_kernel(
     int M, int N, int K, const TA *A, long long lda, const TB *B, long long ldb, int tb, TC *C,
     long long ldc, double alpha, F64Epilogue ep, double *part, int kchunk) {
+    pdl_wait_prev();
+    pdl_launch_next();
     if (ep.skip && *ep.skip) return;
     __shared__ __align__(16) double As[2][F64B_K][F64B_M];
     __shared__ __align__(16) double Bs[2][F64B_K][F64B_N];
@@ -518,6 +522,8 @@ __global__ __launch_bounds__(256, 2) void gemm_f64acc_big_kernel(
 template <typename TC>
 __global__ void f64acc_reduce_kernel(int M, int N, int splits, const double *part, TC *C,
                                      long long ldc, double alpha, F64Epilogue ep) {
+    pdl_wait_prev();
+    pdl_launch_next();
     if (ep.skip && *ep.skip) return;
     const long long total = (long long)M * N;
     const double dg = ep.diag ? (double)*ep.diag : 0.0;
@@ -563,14 +569,15 @@ inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, 
             splits = ceil_div(K, kchunk);
         }
         g2.z = splits;
-        gemm_f64acc_big_kernel<TA, TB, TC><<<g2, 256, 0, s>>>(
-            M, N, K, A, lda, B, ldb, tb, C, ldc, alpha, ep, splits > 1 ? sp.part : nullptr, kchunk);
-        if (int st = launch_status()) return st;
+        if (int st = launch_kernel(gemm_f64acc_big_kernel<TA, TB, TC>, g2, dim3(256), 0, s, true,
+                                   M, N, K, A, lda, B, ldb, tb, C, ldc, alpha, ep,
+                                   splits > 1 ? sp.part : nullptr, kchunk))
+            return st;
         if (splits > 1) {
             const long long total = (long long)M * N;
             const int blocks = (int)((total + 255) / 256 < 4LL * sms ? (total + 255) / 256 : 4LL * sms);
-            f64acc_reduce_kernel<TC><<<blocks, 256, 0, s>>>(M, N, splits, sp.part, C, ldc, alpha, ep);
-            return launch_status();
+            return launch_kernel(f64acc_reduce_kernel<TC>, dim3(blocks), dim3(256), 0, s, true, M, N,
+                                 splits, (const double *)sp.part, C, ldc, alpha, ep);
         }
         return GPTQ_OK;
     }
@@ -590,15 +597,15 @@ inline int gemm_f64acc(int M, int N, int K, const TA *A, long long lda, int ta, 
         splits = ceil_div(K, kchunk);
     }
     grid.z = splits;
-    gemm_f64acc_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, A, lda, ta, B, ldb, tb, C, ldc,
-                                                        alpha, b_upper, ep,
-                                                        splits > 1 ? sp.part : nullptr, kchunk);
-    if (int st = launch_status()) return st;
+    if (int st = launch_kernel(gemm_f64acc_kernel<TA, TB, TC>, grid, dim3(256), 0, s, true, M, N, K,
+                               A, lda, ta, B, ldb, tb, C, ldc, alpha, b_upper, ep,
+                               splits > 1 ? sp.part : nullptr, kchunk))
+        return st;
     if (splits > 1) {
         const long long total = (long long)M * N;
         const int blocks = (int)((total + 255) / 256 < 4LL * sms ? (total + 255) / 256 : 4LL * sms);
-        f64acc_reduce_kernel<TC><<<blocks, 256, 0, s>>>(M, N, splits, sp.part, C, ldc, alpha, ep);
-        return launch_status();
+        return launch_kernel(f64acc_reduce_kernel<TC>, dim3(blocks), dim3(256), 0, s, true, M, N,
+                             splits, (const double *)sp.part, C, ldc, alpha, ep);
     }
     return GPTQ_OK;
 }

@@ -140,6 +140,8 @@ __global__ __launch_bounds__(RES_THREADS) void il_residual_kernel(
     double *part, int *ctl, int phase, double tol, double *resid) {
     const int done_w = phase == 1 ? IL_CTL_DONE1 : IL_CTL_DONE;
     const int count_w = phase == 1 ? IL_CTL_CHECKS1 : IL_CTL_ITERS;
+    pdl_wait_prev();
+    pdl_launch_next();
     if (ctl[done_w]) return;
     extern __shared__ __align__(16) double rsm[];
     double *Qc = rsm;                        // p x 64
@@ -292,14 +294,17 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
     for (int it = 0; it < IL_P1_STEPS; ++it) {
         auto pz = gemm_args<float, float>(n, p, n, H, ldh, 0, w.Y, p, 0, w.Z, p, 1.f, 0.f);
         pz.skip = done1;
+        pz.pdl = 1;
         if (int st = gemm_f32(pz, s)) return st;
         if (it > 0 && it % IL_P1_EVERY == 0) {
             if (int st = gemm_f64acc<float, float, double>(p, p, n, w.Y, p, 1, w.Z, p, 0, w.Tm, p,
                     1.0, s, 0, skip_if(done1), il_split(w))) return st;
             if (int st = sym_eig_top(w.Tm, p, r, w.ev, w.Qr, done1, s)) return st;
-            il_residual_kernel<float><<<rgrid, RES_THREADS, rsmem, s>>>(
-                w.Z, w.Y, w.Qr, w.ev, n, p, r, w.res, w.ctl, 1, IL_P1_TOL, resid);
-            GPTQ_CHECK_LAUNCH();
+            if (int st = launch_kernel(il_residual_kernel<float>, rgrid, dim3(RES_THREADS), rsmem, s,
+                                       true, (const float *)w.Z, (const float *)w.Y,
+                                       (const double *)w.Qr, (const double *)w.ev, n, p, r, w.res,
+                                       w.ctl, 1, IL_P1_TOL, resid))
+                return st;
         }
         if (int st = cholqr_f64<float>(w.Z, w.Y, n, p, w, s, done1)) return st;
     }
@@ -314,9 +319,11 @@ inline int il_top_eigvecs(const float *H, long long ldh, int n, int r, float *V,
         if (int st = gemm_f64acc<float, double, double>(p, p, n, w.Y, p, 1, w.HY, p, 0, w.Tm, p,
                 1.0, s, 0, skip_if(done), il_split(w))) return st;
         if (int st = sym_eig_top(w.Tm, p, r, w.ev, w.Qr, done, s)) return st;
-        il_residual_kernel<double><<<rgrid, RES_THREADS, rsmem, s>>>(
-            w.HY, w.Y, w.Qr, w.ev, n, p, r, w.res, w.ctl, 2, IL_TOL, resid);
-        GPTQ_CHECK_LAUNCH();
+        if (int st = launch_kernel(il_residual_kernel<double>, rgrid, dim3(RES_THREADS), rsmem, s,
+                                   true, (const double *)w.HY, (const float *)w.Y,
+                                   (const double *)w.Qr, (const double *)w.ev, n, p, r, w.res,
+                                   w.ctl, 2, IL_TOL, resid))
+            return st;
     }
     il_finish_kernel<<<1, 32, 0, s>>>(w.ctl);
     GPTQ_CHECK_LAUNCH();

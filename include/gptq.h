@@ -233,12 +233,14 @@ GPTQ_API int gptq_quantize_layer(const void *W, int w_dtype, int64_t m, int64_t 
  * GPTQ_NOALLOC_SCRATCH_BYTES bytes that every device loading the library holds until the
  * process exits. The caller still provides W, U and the outputs, as for
  * gptq_quantize_layer, and the arguments mean the same.
- *   - Limit: gptq_workspace_size(GPTQ_OP_QUANTIZE, m, n, 0, block_size) must not exceed
- *     GPTQ_NOALLOC_SCRATCH_BYTES. That size is m * n floats (the working copy) plus
+ *   - Limit: the scratch, m * n floats (the working copy) plus
  *     2 * m * max(min(n, 1024), block_size) floats (the errors of one 1024-column outer
- *     block, kept as a tf32 high part and its remainder), each part rounded up to 256 bytes;
- *     e.g. 2048 x 6144 fits (exactly), 2048 x 7680 does not. Larger layers get GPTQ_ERR_ARG
- *     and nothing is enqueued.
+ *     block, kept as a tf32 high part and its remainder), each part rounded up to 256 bytes,
+ *     must not exceed GPTQ_NOALLOC_SCRATCH_BYTES; e.g. 2048 x 6144 fits (exactly), 2048 x 7680
+ *     does not. Larger layers get GPTQ_ERR_ARG and nothing is enqueued. (gptq_quantize_layer's
+ *     workspace also holds U's outer-block band split into tf32 pairs, which this entry point
+ *     does without: its tensor-core products split U as they load it. Both round the same
+ *     way, so the outputs are identical.)
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     with that device current; make that first call before any stream capture. The address
  *     is tied to the device's current context: a call made after that context was destroyed

@@ -75,3 +75,52 @@ def test_sweep_bytes_and_roofline():
     assert r["gemm_ms"] == 1.25 and abs(r["column_loop_ms"] - 0.75) < 1e-12
     assert 0 < r["frac"] < 1
     assert "gemm_ms" not in bench.sweep_roofline(layer, 2.0, None)
+
+
+def _layer_digest(rank):
+    """The rank's own layer (weak scaling: an independent layer per rank) through the oracle:
+    (number of weights, code digest, the layer's first weight)."""
+    import hashlib
+    import numpy as np
+    import datagen
+    import oracle
+    L = datagen.tiny(device="cpu", seed=bench.rank_seed("tiny", rank))
+    res = oracle.gptq_layer(L.W.double().numpy(), L.X.double().numpy(), L.bits, L.group_size,
+                            L.lambda_rel)
+    codes = np.ascontiguousarray(res["codes"].astype(np.int64))
+    return L.m * L.n, hashlib.sha256(codes.tobytes()).hexdigest(), float(L.W[0, 0])
+
+
+def _shard_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = _layer_digest(rank)
+        every = [None] * world
+        dist.all_gather_object(every, mine)
+        q.put((rank, every))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_quantize_their_own_layers():
+    """The multi-GPU path shards by layer: each rank quantizes the independent layer its seed
+    names, with no data exchange. Two gloo ranks gather what they computed; each rank's result
+    equals a standalone run of its seed, the two layers differ, and the whole-job unit count is
+    the sum over ranks (bench.py reports world x m x n weights per step)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_shard_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(300)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=5) for _ in range(2))
+    assert got[0] == got[1]                      # both ranks hold the same gathered view
+    every = got[0]
+    alone = [_layer_digest(r) for r in range(2)]
+    assert every == alone                        # rank r computed exactly seed r's layer
+    assert every[0][1] != every[1][1] and every[0][2] != every[1][2]
+    assert sum(e[0] for e in every) == 2 * 256 * 256

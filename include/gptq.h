@@ -162,7 +162,11 @@ GPTQ_API int gptq_kernel_times(gptq_kernel_time *out, int n_out);
  *           strictly lower one may serve as scratch during the call. On return both
  *           triangles hold the symmetric sum.
  *   X       device, k x n row-major calibration chunk; x_dtype GPTQ_BF16 or GPTQ_F32.
- *           The base address must be 16-byte aligned; for GPTQ_BF16, n % 8 == 0.
+ *           The base address must be 16-byte aligned; for GPTQ_BF16, n % 8 == 0. bf16 X runs
+ *           on the bf16 tensor cores with fp32 accumulation; fp32 X on the fp32-accurate
+ *           tensor-core product (tf32 x 3: each operand split into two tf32 parts, three
+ *           products; error ~2^-22 of |x||y| per product) when n % 4 == 0 and n x n is large
+ *           enough, else on an fp32 SIMT kernel.
  *   k, n    k >= 0 tokens (k == 0 is a no-op), 1 <= n <= 65536 features.
  * Call it once per chunk of tokens; chunks are additive and may be of any length.
  */

@@ -413,7 +413,20 @@ static int gptq_hessian_accumulate_body(float *H, const void *X, int x_dtype, in
         }
         return hessian_simt(H, Xb, k, (int)n, s);
     }
-    return hessian_simt(H, static_cast<const float *>(X), k, (int)n, s);
+    // fp32 X: the fp32-accurate tensor-core product (tf32 x 3, both operands split as they
+    // load) over the upper triangle; gemm_f32 itself falls back to the SIMT kernel for small or
+    // unaligned products
+    const auto *Xf = static_cast<const float *>(X);
+    if (std::getenv("GPTQ_FORCE_SIMT_HESSIAN") != nullptr) return hessian_simt(H, Xf, k, (int)n, s);
+    const long long KCH = 1LL << 30;
+    for (long long t0 = 0; t0 < k; t0 += KCH) {
+        const int kc = (int)((k - t0) < KCH ? (k - t0) : KCH);
+        auto p = gemm_args<float, float>((int)n, (int)n, kc, Xf + t0 * n, n, 1, Xf + t0 * n, n, 0, H,
+                                         n, 2.f, 1.f);
+        p.c_upper = 1;
+        if (int st = gemm_f32(p, s)) return st;
+    }
+    return mirror_upper(H, n, n, s);
 }
 
 GPTQ_API int gptq_hessian_accumulate(float *H, const void *X, int x_dtype, int64_t k, int64_t n,

@@ -85,6 +85,28 @@ def test_hessian_tensor_core_path_is_tighter_than_fp32_chain(g, n, k, monkeypatc
     assert e_tc <= REL_H and e_tc <= e_simt
 
 
+@pytest.mark.parametrize("n,k,chunks", [(512, 20000, 2), (1000, 3000, 1), (136, 777, 1)])
+def test_hessian_fp32_x_on_tensor_cores(g, n, k, chunks, monkeypatch):
+    """fp32 X with n % 4 == 0 runs on the fp32-accurate tensor-core product (tf32 x 3) over the
+    upper triangle (n = 136 is small enough to take the SIMT kernel inside it); the forced SIMT
+    path is a plain fp32 chain. Both against the oracle, chunks additive."""
+    X = torch.from_numpy(_spd_from_data(n, k, 5 * n + k)).float().to(DEV)
+    Href = oracle.hessian(np64(X))
+    bounds = np.linspace(0, k, chunks + 1).astype(int)
+    H_tc = torch.zeros(n, n, device=DEV)
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        g.gptq_hessian_accumulate(H_tc, X[a:b].contiguous())
+    g.gptq_sync_status()
+    monkeypatch.setenv("GPTQ_FORCE_SIMT_HESSIAN", "1")
+    H_simt = torch.zeros(n, n, device=DEV)
+    g.gptq_hessian_accumulate(H_simt, X)
+    g.gptq_sync_status()
+    e_tc, e_simt = rel_fro(np64(H_tc), Href), rel_fro(np64(H_simt), Href)
+    print(f"fp32 X n={n} k={k}: tensor-core rel err {e_tc:.2e}, SIMT rel err {e_simt:.2e}")
+    assert torch.equal(H_tc, H_tc.t())
+    assert e_tc <= REL_H and e_simt <= REL_H
+
+
 def test_hessian_bounded_wait_reports_timeout_and_device_stays_usable(g, monkeypatch):
     """A wait that nothing will ever satisfy (test hook) gives up after the limit, reports
     GPTQ_ERR_TIMEOUT through the status word, and the next call works normally."""

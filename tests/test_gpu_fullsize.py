@@ -15,7 +15,7 @@ from gpu_parity import REL_H, REL_LOSS, REL_SCALE, check_replay, np64, rel_fro, 
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-ROWS = np.arange(0, 2048, 64)       # 32 rows spread over the layer
+ROWS = np.arange(0, 2048, 16)       # 128 rows spread over the layer
 
 
 @pytest.fixture(scope="module")

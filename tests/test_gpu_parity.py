@@ -226,6 +226,10 @@ SWEEP_CASES = [
     (48, 256, 5, 64, 64, torch.float32),
     (40, 512, 6, 128, 128, torch.bfloat16),
     (36, 256, 7, 32, 32, torch.float32),
+    # groups shorter than the column loop's 16-column slots: boundaries inside a slot
+    (40, 256, 4, 8, 64, torch.float32),
+    (24, 128, 3, 4, 32, torch.float32),
+    (20, 256, 2, 2, 128, torch.bfloat16),
     # 300 rows: the tensor-core lazy updates' last 32-row slices cross the matrix edge
     (300, 640, 4, 128, 128, torch.float32),
     # several 1024-column outer blocks of the two-level lazy update

@@ -62,7 +62,7 @@ __device__ __forceinline__ void grid_from_range(float mn, float mx, float fmaxq,
     z = fminf(fmaxf(rintf(__fdiv_rn(-mn, s)), 0.f), fmaxq);
 }
 
-constexpr int COLLOOP_THREADS = 128;
+constexpr int COLLOOP_THREADS = 64;
 
 // One warp = 32 / LPR rows; the LPR = B / CPL lanes of a row each hold CPL (16) consecutive
 // columns of the panel in registers (lane k of the row: columns CPL k .. CPL k + CPL-1, "slot"
